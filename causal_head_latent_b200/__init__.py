@@ -1,0 +1,206 @@
+"""Gated MLA hot path for NVIDIA B200 (sm_100a): thin Python binding of libgmla.so.
+
+Every function below marshals arguments for the C ABI of the same name
+(include/gmla.h) and nothing else: all arithmetic runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  If the
+library is missing this module raises ImportError -- there is no fallback.
+
+Layer (the "Gated MLA" problem page): C = X W_c^T, Q = X W_q^T, K = C W_k^T,
+V = C W_v^T, per-head causal softmax attention, heads joined, gate
+sigmoid(X W_g^T), output projection W_o^T.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "GmlaError", "lib", "library_path",
+    "gmla_latent_project", "gmla_latent_project_workspace_size",
+    "gmla_attend_prefill", "gmla_attend_decode", "gmla_attend_decode_workspace_size",
+    "gmla_gate_out", "gmla_gate_out_workspace_size", "gmla_get_device_status", "gmla_status_string",
+    "gmla_version", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libgmla.so")
+
+STATUS = {0: "GMLA_OK", 1: "GMLA_ERR_ARG", 2: "GMLA_ERR_UNSUPPORTED", 3: "GMLA_ERR_CUDA",
+          4: "GMLA_ERR_TIMEOUT", 5: "GMLA_ERR_WORKSPACE"}
+
+if not os.path.exists(library_path):
+    raise ImportError(f"libgmla.so not built ({library_path}); run `python -m causal_head_latent_b200.build`")
+
+lib = ctypes.CDLL(library_path)
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+_st = ctypes.c_int
+_i64x3 = ctypes.c_int64 * 3
+
+lib.gmla_latent_project.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _i64, _i64,
+                                    _p, _p, _p, _sz, _p]
+lib.gmla_latent_project.restype = _st
+lib.gmla_latent_project_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
+lib.gmla_latent_project_workspace_size.restype = _sz
+lib.gmla_attend_prefill.argtypes = [_p, _i64x3, _p, _i64x3, _p, _i64x3, _i64, _i64, _i64, _i64, _i64,
+                                    ctypes.c_int, ctypes.c_float, _p, _p, _i64x3, _p, _p, _p]
+lib.gmla_attend_prefill.restype = _st
+lib.gmla_attend_decode.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p, _p, _p,
+                                   _p, _sz, _p]
+lib.gmla_attend_decode.restype = _st
+lib.gmla_attend_decode_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
+lib.gmla_attend_decode_workspace_size.restype = _sz
+lib.gmla_gate_out.argtypes = [_p, _p, _p, _i64, _i64, _p, _p, _sz, _p]
+lib.gmla_gate_out.restype = _st
+lib.gmla_gate_out_workspace_size.argtypes = [_i64, _i64]
+lib.gmla_gate_out_workspace_size.restype = _sz
+lib.gmla_get_device_status.argtypes = [_p]
+lib.gmla_get_device_status.restype = _st
+lib.gmla_status_string.argtypes = [_st]
+lib.gmla_status_string.restype = ctypes.c_char_p
+lib.gmla_version.argtypes = []
+lib.gmla_version.restype = ctypes.c_int
+
+
+class GmlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({gmla_status_string(code)})")
+
+
+def _check(code: int, where: str) -> int:
+    if code != 0:
+        raise GmlaError(code, where)
+    return code
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    return t.data_ptr()
+
+
+def _bf16(t, name):
+    if t is not None and t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def gmla_status_string(code: int) -> str:
+    return lib.gmla_status_string(code).decode()
+
+
+def gmla_version() -> int:
+    return lib.gmla_version()
+
+
+def gmla_get_device_status(stream=None, raise_on_error: bool = True) -> int:
+    code = lib.gmla_get_device_status(_stream(stream))
+    return _check(code, "gmla_get_device_status") if raise_on_error else code
+
+
+def gmla_latent_project_workspace_size(B, T, d_model, d_c) -> int:
+    return lib.gmla_latent_project_workspace_size(B, T, d_model, d_c)
+
+
+def gmla_latent_project(X, W_q, W_g, W_c, W_k, W_v, Q=None, G=None, C=None, cache_len_max=None, cache_pos=0,
+                        K=None, V=None, workspace=None, stream=None, check=True):
+    """X [B, T, d_model]; C [B, cache_len_max, d_c] (rows cache_pos..cache_pos+T-1 written)."""
+    for n, t in (("X", X), ("W_q", W_q), ("W_g", W_g), ("W_c", W_c), ("W_k", W_k), ("W_v", W_v),
+                 ("Q", Q), ("G", G), ("C", C), ("K", K), ("V", V)):
+        _bf16(t, n)
+    B, T, d = X.shape
+    d_c = W_c.shape[0] if W_c is not None else (C.shape[-1] if C is not None else 0)
+    if cache_len_max is None:
+        cache_len_max = C.shape[1] if C is not None else T
+    wp, wb = _ws(workspace)
+    code = lib.gmla_latent_project(_ptr(X), B, T, d, _ptr(W_q), _ptr(W_g), _ptr(W_c), d_c, _ptr(W_k), _ptr(W_v),
+                                   _ptr(Q), _ptr(G), _ptr(C), cache_len_max, cache_pos, _ptr(K), _ptr(V), wp, wb,
+                                   _stream(stream))
+    return _check(code, "gmla_latent_project") if check else code
+
+
+def _bthd_strides(t, layout):
+    """(batch, token, head) element strides of a 4-D tensor in layout 'bthd' or 'bhtd'."""
+    if t.stride(-1) != 1:
+        raise ValueError("head dimension must be contiguous")
+    s = t.stride()
+    return _i64x3(s[0], s[1], s[2]) if layout == "bthd" else _i64x3(s[0], s[2], s[1])
+
+
+def gmla_attend_prefill(Q, K, V, O, causal=True, scale=0.0, G=None, lse=None, weights=None, layout="bthd",
+                        stream=None, check=True):
+    """Q, O [B,Tq,H,D] (or [B,H,Tq,D] with layout='bhtd'); K, V [B,Tk,H,D]; G [B,Tq,H*D] or None."""
+    for n, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("G", G)):
+        _bf16(t, n)
+    if layout == "bthd":
+        B, Tq, H, D = Q.shape
+        Tk = K.shape[1]
+    else:
+        B, H, Tq, D = Q.shape
+        Tk = K.shape[2]
+    if lse is not None and lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
+    if weights is not None and weights.dtype != torch.float32:
+        raise TypeError("weights must be float32")
+    code = lib.gmla_attend_prefill(_ptr(Q), _bthd_strides(Q, layout), _ptr(K), _bthd_strides(K, layout), _ptr(V),
+                                   _bthd_strides(V, layout), B, H, Tq, Tk, D, int(bool(causal)), float(scale),
+                                   _ptr(G), _ptr(O), _bthd_strides(O, layout), _ptr(lse), _ptr(weights),
+                                   _stream(stream))
+    return _check(code, "gmla_attend_prefill") if check else code
+
+
+def gmla_attend_decode_workspace_size(B, L, H, d_c) -> int:
+    return lib.gmla_attend_decode_workspace_size(B, L, H, d_c)
+
+
+def gmla_attend_decode(Q, C, L, W_k, W_v, O, num_heads, scale=0.0, G=None, weights=None, workspace=None,
+                       stream=None, check=True):
+    """Q, O, G [B, H*D]; C [B, cache_len_max, d_c]; rows 0..L-1 visible."""
+    for n, t in (("Q", Q), ("C", C), ("W_k", W_k), ("W_v", W_v), ("O", O), ("G", G)):
+        _bf16(t, n)
+    B, d = Q.shape
+    H = int(num_heads)
+    D = d // H
+    _, Lmax, d_c = C.shape
+    wp, wb = _ws(workspace)
+    code = lib.gmla_attend_decode(_ptr(Q), _ptr(C), B, Lmax, L, H, D, d_c, _ptr(W_k), _ptr(W_v), float(scale),
+                                  _ptr(G), _ptr(O), _ptr(weights), wp, wb, _stream(stream))
+    return _check(code, "gmla_attend_decode") if check else code
+
+
+def gmla_gate_out_workspace_size(M, d_model) -> int:
+    return lib.gmla_gate_out_workspace_size(M, d_model)
+
+
+def gmla_gate_out(O, W_o, Y, G=None, workspace=None, stream=None, check=True):
+    """O, Y [M, d_model] (any leading shape flattened); W_o [d_model, d_model]."""
+    for n, t in (("O", O), ("W_o", W_o), ("Y", Y), ("G", G)):
+        _bf16(t, n)
+    d = O.shape[-1]
+    M = O.numel() // d
+    wp, wb = _ws(workspace)
+    code = lib.gmla_gate_out(_ptr(O), _ptr(G), _ptr(W_o), M, d, _ptr(Y), wp, wb, _stream(stream))
+    return _check(code, "gmla_gate_out") if check else code

@@ -1,0 +1,358 @@
+// C-ABI entry points of libgmla.so (declared in include/gmla.h).
+//
+// Every entry point checks its arguments on the host, builds the TMA tensor
+// maps it needs, and launches on the caller's stream.  Nothing is allocated
+// per call: scratch lives in a caller workspace.  A device status word
+// (one per device) collects in-kernel timeouts; gmla_get_device_status reads
+// and clears it.
+#include <math.h>
+#include <mutex>
+
+#include "../../include/gmla.h"
+#include "internal.h"
+
+namespace gmla {
+
+__device__ unsigned g_status_word;
+
+static constexpr int kMaxDevices = 64;
+static unsigned *g_status_ptr[kMaxDevices];
+static int g_num_sms[kMaxDevices];
+static std::mutex g_mu;
+
+static int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+// Per-device set-up: the status word's device address and the SM count.
+static bool device_setup(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_status_ptr[dev]) return true;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return false;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  g_num_sms[dev] = sms;
+  g_status_ptr[dev] = static_cast<unsigned *>(p);
+  return true;
+}
+
+int num_sms() {
+  const int d = current_device();
+  return (d >= 0 && d < kMaxDevices && g_num_sms[d] > 0) ? g_num_sms[d] : 148;
+}
+
+static unsigned *status_ptr() {
+  const int d = current_device();
+  if (!device_setup(d)) return nullptr;
+  return g_status_ptr[d];
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tiled map with 128-byte swizzle.  dims/strides in elements, dim 0 innermost (contiguous).
+static bool make_map(CUtensorMap *m, const void *base, int rank, const long long *dims, const long long *strides,
+                     const unsigned *box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = (cuuint64_t)dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = (cuuint64_t)strides[i] * 2;  // bytes, dims 1..rank-1
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace gmla
+
+using namespace gmla;
+
+extern "C" {
+
+int gmla_version(void) { return 100; }
+
+const char *gmla_status_string(gmla_status s) {
+  switch (s) {
+    case GMLA_OK: return "ok";
+    case GMLA_ERR_ARG: return "invalid argument";
+    case GMLA_ERR_UNSUPPORTED: return "unsupported size or option";
+    case GMLA_ERR_CUDA: return "CUDA error";
+    case GMLA_ERR_TIMEOUT: return "bounded in-kernel wait timed out";
+    case GMLA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+gmla_status gmla_get_device_status(gmla_stream_t stream) {
+  unsigned *sp = status_ptr();
+  if (!sp) return GMLA_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GMLA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, sp, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return GMLA_ERR_CUDA;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(sp, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return GMLA_ERR_CUDA;
+  }
+  if (v & kStatusTimeout) return GMLA_ERR_TIMEOUT;
+  if (v) return GMLA_ERR_CUDA;
+  return GMLA_OK;
+}
+
+// ------------------------------------------------------------------ projections
+
+size_t gmla_latent_project_workspace_size(int64_t B, int64_t T, int64_t d_model, int64_t d_c) {
+  (void)B; (void)T; (void)d_model; (void)d_c;
+  return 0;
+}
+
+gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model, const gmla_bf16 *W_q,
+                                const gmla_bf16 *W_g, const gmla_bf16 *W_c, int64_t d_c, const gmla_bf16 *W_k,
+                                const gmla_bf16 *W_v, gmla_bf16 *Q, gmla_bf16 *G, gmla_bf16 *C,
+                                int64_t cache_len_max, int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V,
+                                void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
+  (void)workspace; (void)workspace_bytes;
+  if (!X || B <= 0 || T <= 0 || d_model <= 0 || d_c <= 0) return GMLA_ERR_ARG;
+  if ((Q && !W_q) || (G && !W_g) || (C && !W_c) || (K && !W_k) || (V && !W_v)) return GMLA_ERR_ARG;
+  if ((K || V) && !C) return GMLA_ERR_ARG;
+  if (C && (cache_pos < 0 || cache_len_max <= 0 || cache_pos + T > cache_len_max)) return GMLA_ERR_ARG;
+  const void *ptrs[] = {X, W_q, W_g, W_c, W_k, W_v, Q, G, C, K, V};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (d_model % 128 != 0 || d_c % 64 != 0) return GMLA_ERR_UNSUPPORTED;
+  if (B * T > 0x7fffffffLL || cache_len_max > 0x7fffffffLL || B > 65535) return GMLA_ERR_UNSUPPORTED;
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long M = B * T;
+
+  // [Q | G | C] = X [W_q; W_g; W_c]^T
+  {
+    GemmArgs ga{};
+    CUtensorMap tmA, tmB[3];
+    const long long dA[3] = {d_model, M, 1}, sA[2] = {d_model, M * d_model};
+    const unsigned bA[3] = {64, 128, 1};
+    if (!make_map(&tmA, X, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+    ga.a_rows = (int)M;
+    ga.a_batches = 1;
+    ga.a_row0 = 0;
+    ga.K = (int)d_model;
+    ga.status = st;
+    int np = 0;
+    const gmla_bf16 *Ws[3] = {W_q, W_g, W_c};
+    gmla_bf16 *Os[3] = {Q, G, C};
+    for (int i = 0; i < 3; ++i) {
+      if (!Os[i]) continue;
+      const long long N = i == 2 ? d_c : d_model;
+      const long long dB[2] = {d_model, N}, sB[1] = {d_model};
+      const unsigned bB[2] = {64, 256};
+      if (!make_map(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+      GemmOut &o = ga.prob[np];
+      o.out = Os[i];
+      o.N = (int)N;
+      if (i == 2) {  // latent rows go to cache rows [cache_pos, cache_pos + T) of each batch
+        o.rows_per_b = T;
+        o.sb = cache_len_max * d_c;
+        o.st = d_c;
+        o.off = cache_pos * d_c;
+      } else {
+        o.rows_per_b = M;
+        o.sb = 0;
+        o.st = d_model;
+        o.off = 0;
+      }
+      ++np;
+    }
+    ga.n_problems = np;
+    if (np > 0 && launch_gemm(tmA, tmB, ga, s) != 0) return GMLA_ERR_CUDA;
+  }
+  // [K | V] = C [W_k; W_v]^T, reading the bf16 latents just written to the cache
+  if (K || V) {
+    GemmArgs ga{};
+    CUtensorMap tmA, tmB[3];
+    const long long dA[3] = {d_c, cache_pos + T, B}, sA[2] = {d_c, cache_len_max * d_c};
+    const unsigned bA[3] = {64, 128, 1};
+    if (!make_map(&tmA, C, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+    ga.a_rows = (int)T;
+    ga.a_batches = (int)B;
+    ga.a_row0 = (int)cache_pos;
+    ga.K = (int)d_c;
+    ga.status = st;
+    int np = 0;
+    const gmla_bf16 *Ws[2] = {W_k, W_v};
+    gmla_bf16 *Os[2] = {K, V};
+    for (int i = 0; i < 2; ++i) {
+      if (!Os[i]) continue;
+      const long long dB[2] = {d_c, d_model}, sB[1] = {d_c};
+      const unsigned bB[2] = {64, 256};
+      if (!make_map(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+      GemmOut &o = ga.prob[np];
+      o.out = Os[i];
+      o.N = (int)d_model;
+      o.rows_per_b = M;
+      o.sb = 0;
+      o.st = d_model;
+      o.off = 0;
+      ++np;
+    }
+    ga.n_problems = np;
+    if (launch_gemm(tmA, tmB, ga, s) != 0) return GMLA_ERR_CUDA;
+  }
+  return GMLA_OK;
+}
+
+// ------------------------------------------------------------------ attention over explicit Q, K, V
+
+gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_strides[3], const gmla_bf16 *K,
+                                const int64_t k_strides[3], const gmla_bf16 *V, const int64_t v_strides[3],
+                                int64_t B, int64_t H, int64_t Tq, int64_t Tk, int64_t D_h, int causal, float scale,
+                                const gmla_bf16 *G, gmla_bf16 *O, const int64_t o_strides[3], float *lse,
+                                float *weights, gmla_stream_t stream) {
+  if (!Q || !K || !V || !O || !q_strides || !k_strides || !v_strides || !o_strides) return GMLA_ERR_ARG;
+  if (B <= 0 || H <= 0 || Tq < 0 || Tk <= 0 || Tq > Tk || D_h <= 0) return GMLA_ERR_ARG;
+  if (causal != 0 && causal != 1) return GMLA_ERR_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (G && !aligned16(G))) return GMLA_ERR_ARG;
+  for (int i = 0; i < 3; ++i) {
+    if (q_strides[i] <= 0 || k_strides[i] <= 0 || v_strides[i] <= 0 || o_strides[i] <= 0) return GMLA_ERR_ARG;
+    if (q_strides[i] % 8 || k_strides[i] % 8 || v_strides[i] % 8 || o_strides[i] % 8) return GMLA_ERR_ARG;
+  }
+  if (D_h != 128) return GMLA_ERR_UNSUPPORTED;
+  if (B > 0xffff || H > 0xffff || Tk > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  if (Tq == 0) return GMLA_OK;
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D_h);
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (Tq <= 4) {
+    RowsArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.G = G; a.O = O;
+    for (int i = 0; i < 3; ++i) {
+      a.qs[i] = q_strides[i]; a.ks[i] = k_strides[i]; a.vs[i] = v_strides[i]; a.os[i] = o_strides[i];
+    }
+    a.lse = lse; a.weights = weights;
+    a.B = (int)B; a.H = (int)H; a.Tq = (int)Tq; a.Tk = (int)Tk; a.causal = causal;
+    a.scale = scale; a.status = st;
+    return launch_attn_rows(a, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+  }
+
+  CUtensorMap tq, tk, tv;
+  const unsigned box[4] = {64, 128, 1, 1};
+  {
+    const long long d[4] = {128, Tq, H, B}, sd[3] = {q_strides[1], q_strides[2], q_strides[0]};
+    if (!make_map(&tq, Q, 4, d, sd, box)) return GMLA_ERR_CUDA;
+  }
+  {
+    const long long d[4] = {128, Tk, H, B}, sd[3] = {k_strides[1], k_strides[2], k_strides[0]};
+    if (!make_map(&tk, K, 4, d, sd, box)) return GMLA_ERR_CUDA;
+  }
+  {
+    const long long d[4] = {128, Tk, H, B}, sd[3] = {v_strides[1], v_strides[2], v_strides[0]};
+    if (!make_map(&tv, V, 4, d, sd, box)) return GMLA_ERR_CUDA;
+  }
+  PrefillArgs a{};
+  a.G = G; a.O = O;
+  for (int i = 0; i < 3; ++i) a.o_strides[i] = o_strides[i];
+  a.lse = lse; a.weights = weights;
+  a.B = (int)B; a.H = (int)H; a.Tq = (int)Tq; a.Tk = (int)Tk; a.causal = causal;
+  a.scale = scale; a.status = st;
+  return launch_attn_prefill(tq, tk, tv, a, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ decode over the latent cache
+
+size_t gmla_attend_decode_workspace_size(int64_t B, int64_t L, int64_t H, int64_t d_c) {
+  if (B <= 0 || L <= 0 || H <= 0 || d_c <= 0) return 0;
+  return latent_workspace_bytes(B, L, H, d_c);
+}
+
+gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B, int64_t cache_len_max, int64_t L,
+                               int64_t H, int64_t D_h, int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v,
+                               float scale, const gmla_bf16 *G, gmla_bf16 *O, float *weights, void *workspace,
+                               size_t workspace_bytes, gmla_stream_t stream) {
+  if (!Q || !C || !W_k || !W_v || !O) return GMLA_ERR_ARG;
+  if (B <= 0 || H <= 0 || D_h <= 0 || d_c <= 0 || L < 1 || cache_len_max < L) return GMLA_ERR_ARG;
+  const void *ptrs[] = {Q, C, W_k, W_v, G, O, workspace};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (D_h != 128 || d_c % 64 != 0 || d_c > 512) return GMLA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || L > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  const size_t need = latent_workspace_bytes(B, L, H, d_c);
+  if (!workspace || workspace_bytes < need) return GMLA_ERR_WORKSPACE;
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D_h);
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  LatentArgs a{};
+  a.Q = Q; a.C = C; a.Wk = W_k; a.Wv = W_v; a.G = G; a.O = O; a.weights = weights;
+  a.cache_len_max = cache_len_max;
+  a.B = (int)B; a.L = (int)L; a.H = (int)H; a.dc = (int)d_c;
+  a.scale = scale; a.workspace = workspace; a.status = st;
+  return launch_attend_latent(a, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ output projection
+
+size_t gmla_gate_out_workspace_size(int64_t M, int64_t d_model) {
+  (void)M; (void)d_model;
+  return 0;
+}
+
+gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M, int64_t d_model,
+                          gmla_bf16 *Y, void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
+  (void)workspace; (void)workspace_bytes;
+  if (!O || !W_o || !Y || M <= 0 || d_model <= 0) return GMLA_ERR_ARG;
+  if (!aligned16(O) || !aligned16(W_o) || !aligned16(Y)) return GMLA_ERR_ARG;
+  if (G) return GMLA_ERR_UNSUPPORTED;
+  if (d_model % 128 != 0 || M > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  GemmArgs ga{};
+  CUtensorMap tmA, tmB[3];
+  const long long dA[3] = {d_model, M, 1}, sA[2] = {d_model, M * d_model};
+  const unsigned bA[3] = {64, 128, 1};
+  if (!make_map(&tmA, O, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+  const long long dB[2] = {d_model, d_model}, sB[1] = {d_model};
+  const unsigned bB[2] = {64, 256};
+  if (!make_map(&tmB[0], W_o, 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+  ga.a_rows = (int)M;
+  ga.a_batches = 1;
+  ga.a_row0 = 0;
+  ga.K = (int)d_model;
+  ga.status = st;
+  ga.n_problems = 1;
+  ga.prob[0].out = Y;
+  ga.prob[0].N = (int)d_model;
+  ga.prob[0].rows_per_b = M;
+  ga.prob[0].sb = 0;
+  ga.prob[0].st = d_model;
+  ga.prob[0].off = 0;
+  return launch_gemm(tmA, tmB, ga, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
+}  // extern "C"

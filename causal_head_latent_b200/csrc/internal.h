@@ -1,0 +1,80 @@
+// Internal launch interfaces between the C-ABI layer (gmla_api.cu) and the
+// kernels.  Not part of the public ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gmla {
+
+// Device status word bits (read back by gmla_get_device_status).
+constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusBadIndex = 2u;
+
+// ---------------------------------------------------------------- prefill attention
+struct PrefillArgs {
+  const uint16_t *G;  // optional gate logits [B, Tq, H*128]
+  uint16_t *O;
+  long long o_strides[3];
+  float *lse;
+  float *weights;
+  int B, H, Tq, Tk, causal;
+  float scale;
+  unsigned *status;
+};
+// tmQ/tmK/tmV: 4-D maps (D=128, T, H, B), bf16, box (64, 128, 1, 1), 128-byte swizzle.
+int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                        const PrefillArgs &a, cudaStream_t stream);
+size_t attn_prefill_smem_bytes();
+
+// ---------------------------------------------------------------- few-query attention (decode over explicit K/V)
+struct RowsArgs {
+  const uint16_t *Q, *K, *V, *G;
+  long long qs[3], ks[3], vs[3], os[3];
+  uint16_t *O;
+  float *lse;
+  float *weights;
+  int B, H, Tq, Tk, causal;
+  float scale;
+  unsigned *status;
+};
+int launch_attn_rows(const RowsArgs &a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- tcgen05 GEMM  D = A B^T
+// Output row mapping: global row m -> element offset
+//   (m / rows_per_b) * sb + (m % rows_per_b) * st + off
+struct GemmOut {
+  uint16_t *out;
+  long long rows_per_b, sb, st, off;
+  int N;
+};
+struct GemmArgs {
+  int a_rows;        // rows per batch of A (rows of the A map's dimension 1 that belong to the problem)
+  int a_batches;     // batches (A map dimension 2)
+  int a_row0;        // first row coordinate in the A map
+  int K;
+  int n_problems;    // 1..3, all share A
+  GemmOut prob[3];
+  unsigned *status;
+};
+// tmA: 3-D map (K, rows, batches), box (64, 128, 1); tmB[i]: 2-D map (K, N_i), box (64, 256).
+int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode over the latent cache
+struct LatentArgs {
+  const uint16_t *Q, *C, *Wk, *Wv, *G;
+  uint16_t *O;
+  float *weights;
+  long long cache_len_max;
+  int B, L, H, dc;
+  float scale;
+  void *workspace;
+  unsigned *status;
+};
+int launch_attend_latent(const LatentArgs &a, cudaStream_t stream);
+size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc);
+
+int num_sms();
+
+}  // namespace gmla

@@ -1,0 +1,190 @@
+/*
+ * gmla.h -- C ABI of the Gated MLA (gated multi-head latent attention) hot path
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The layer (the "Gated MLA" problem page, sections "Start from familiar
+ * attention", "Split attention into heads" and "The channel-wise output
+ * gate") is
+ *
+ *     C = X W_c^T,  Q = X W_q^T,  K = C W_k^T,  V = C W_v^T,
+ *     per head h:  A_h = softmax(Q_h K_h^T / sqrt(D_h) + M),  O_h = A_h V_h,
+ *     O = [O_1 | ... | O_H]                      (heads joined, not summed)
+ *     Y = (sigmoid(X W_g^T) (.) O) W_o^T
+ *
+ * with the causal mask M[t,s] = 0 for s <= t and -inf for s > t ("Kimi K2 -
+ * Construct causal mask"), the softmax taken over keys in float32 ("Kimi K3 -
+ * Softmax over keys") and no positional encoding.  The latent C is the only
+ * cached tensor.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor is bfloat16 (gmla_bf16 holds the raw 16-bit pattern) unless
+ *    stated otherwise; debug outputs are float32.
+ *  - Every pointer is a DEVICE pointer on the current CUDA device, except where
+ *    a comment says host.  The caller owns every buffer.  The library never
+ *    allocates memory in a call; scratch comes from a caller workspace whose
+ *    size the matching *_workspace_size function returns.
+ *  - Inputs are never written.  The latent cache C is the one in/out buffer:
+ *    gmla_latent_project writes only rows [cache_pos, cache_pos + T).
+ *  - Weights use the nn.Linear orientation [out_features, in_features]:
+ *    W_q, W_g, W_o [d_model, d_model]; W_c [d_c, d_model]; W_k, W_v [d_model, d_c].
+ *  - Head h owns channels [h*D_h, (h+1)*D_h) of model width (D_h = d_model / H).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and return before the GPU work ends.  Only
+ *    gmla_get_device_status synchronises.
+ *  - Arguments are checked on the host before any launch; a bad argument
+ *    returns GMLA_ERR_ARG and launches nothing.  Device pointers must be
+ *    16-byte aligned and row strides multiples of 8 elements.
+ *  - Supported sizes: D_h = 128 (the pages fix 96 heads of width 128), d_c a
+ *    multiple of 64, d_model = 128 * H.  Other sizes return
+ *    GMLA_ERR_UNSUPPORTED.
+ *  - Every wait inside a kernel is bounded; a wait that runs out records
+ *    GMLA_ERR_TIMEOUT in a device status word read by gmla_get_device_status.
+ */
+#ifndef GMLA_H
+#define GMLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GMLA_API __attribute__((visibility("default")))
+#else
+#define GMLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GMLA_OK = 0,
+    GMLA_ERR_ARG = 1,         /* invalid argument (null, shape, alignment, causal flag) */
+    GMLA_ERR_UNSUPPORTED = 2, /* valid but outside the sizes this library implements */
+    GMLA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
+    GMLA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (device status word) */
+    GMLA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than required */
+} gmla_status;
+
+typedef uint16_t gmla_bf16; /* raw bfloat16 bits */
+typedef void *gmla_stream_t; /* a cudaStream_t */
+
+/*
+ * gmla_latent_project -- the projections of the hidden states.
+ * "Gated MLA" page, sections "Start from familiar attention" (C = X W_c^T,
+ * K = C W_k^T, V = C W_v^T; queries come straight from the hidden states,
+ * read as Q = X W_q^T) and "The channel-wise output gate" (gate logits
+ * G = X W_g^T); implementation-order steps 1, 2 and the gate of step 6.
+ *
+ *  X       [B, T, d_model]                      hidden states (input)
+ *  W_q, W_g [d_model, d_model]; W_c [d_c, d_model]; W_k, W_v [d_model, d_c]
+ *  Q, G    [B, T, d_model]  outputs, may be NULL to skip (then the matching
+ *                           weight may be NULL too)
+ *  C       latent cache [B, cache_len_max, d_c]; row cache_pos + t of batch b
+ *          receives the latent of token (b, t).  Prefill: cache_pos = 0;
+ *          decode of one new token: T = 1, cache_pos = L - 1.
+ *          cache_pos + T <= cache_len_max.  Required when K or V is requested.
+ *  K, V    [B, T, d_model] outputs, may be NULL.  They are expanded from the
+ *          bfloat16 latents just written to C.
+ *  workspace / workspace_bytes: scratch of at least
+ *          gmla_latent_project_workspace_size(B, T, d_model, d_c) bytes
+ *          (may be NULL when that size is 0).
+ * Returns GMLA_ERR_ARG for null required pointers, d_model != 128*H shapes
+ * that are not multiples of 128, cache_pos + T > cache_len_max, or
+ * misalignment; GMLA_ERR_WORKSPACE for a short workspace.
+ */
+GMLA_API gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model,
+                                const gmla_bf16 *W_q, const gmla_bf16 *W_g, const gmla_bf16 *W_c,
+                                int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v,
+                                gmla_bf16 *Q, gmla_bf16 *G, gmla_bf16 *C, int64_t cache_len_max,
+                                int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V, void *workspace,
+                                size_t workspace_bytes, gmla_stream_t stream);
+GMLA_API size_t gmla_latent_project_workspace_size(int64_t B, int64_t T, int64_t d_model, int64_t d_c);
+
+/*
+ * gmla_attend_prefill -- per-head scaled dot-product attention over explicit
+ * Q, K, V, with the causal mask and float32 softmax over keys, optionally
+ * followed by the channel gate.  "Gated MLA" page, "Start from familiar
+ * attention" (A = softmax(QK^T/sqrt(D_h) + M), context A V) and steps 3-5;
+ * "Kimi K3 - Softmax over keys" (weights of visible keys sum to one, blocked
+ * keys weigh zero, P cast to the input type before P V); "Kimi K2 - Construct
+ * causal mask" (positions numbered from the cached length).
+ *
+ *  Q       [B, Tq, H, D_h] as addressed by q_strides; K, V [B, Tk, H, D_h].
+ *          *_strides[0..2] are the element strides of batch, token and head;
+ *          the D_h elements of one head are contiguous.  Both [B,T,H,D] and
+ *          [B,H,T,D] layouts are expressible.
+ *  Tq <= Tk: query t sits at absolute position Tk - Tq + t and, when causal,
+ *          sees keys s <= Tk - Tq + t.  causal must be 0 or 1.
+ *  scale   softmax scale; <= 0 selects 1/sqrt(D_h).
+ *  G       optional gate logits [B, Tq, H*D_h] (contiguous); when given, O
+ *          receives sigmoid(G) (.) O.
+ *  O       output [B, Tq, H, D_h] as addressed by o_strides (bfloat16).
+ *  lse     optional float32 [B, H, Tq]: natural log of sum_s exp(scale * q.k_s)
+ *          over visible keys.
+ *  weights optional float32 [B, H, Tq, Tk] debug softmax weights (before the
+ *          bfloat16 cast), zero for blocked keys.  Slow; for checks only.
+ */
+GMLA_API gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_strides[3],
+                                const gmla_bf16 *K, const int64_t k_strides[3],
+                                const gmla_bf16 *V, const int64_t v_strides[3], int64_t B, int64_t H,
+                                int64_t Tq, int64_t Tk, int64_t D_h, int causal, float scale,
+                                const gmla_bf16 *G, gmla_bf16 *O, const int64_t o_strides[3],
+                                float *lse, float *weights, gmla_stream_t stream);
+
+/*
+ * gmla_attend_decode -- one new query per sequence over the latent cache.
+ * Same mathematics as gmla_attend_prefill with Tq = 1 over K = C W_k^T and
+ * V = C W_v^T ("Gated MLA" page, "Start from familiar attention"), evaluated
+ * without rebuilding K or V: by associativity q_h . (W_k^(h) c_s) =
+ * (W_k^(h)T q_h) . c_s and sum_s a_s W_v^(h) c_s = W_v^(h) sum_s a_s c_s, so
+ * the kernel streams only the d_c-wide latents, each read once for all heads.
+ * The key range is split over thread blocks and the partial softmax states are
+ * merged exactly (log-sum-exp).
+ *
+ *  Q       [B, H*D_h] queries of the new tokens (from gmla_latent_project, T=1)
+ *  C       latent cache [B, cache_len_max, d_c]; rows 0..L-1 are visible (the
+ *          new token's own latent at row L-1 included), 1 <= L <= cache_len_max.
+ *  W_k, W_v [H*D_h, d_c]
+ *  scale   <= 0 selects 1/sqrt(D_h)
+ *  G       optional gate logits [B, H*D_h]; when given, O = sigmoid(G) (.) O
+ *  O       output [B, H*D_h]
+ *  weights optional float32 [B, H, L] debug softmax weights
+ *  workspace >= gmla_attend_decode_workspace_size(B, L, H, d_c) bytes
+ */
+GMLA_API gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B,
+                               int64_t cache_len_max, int64_t L, int64_t H, int64_t D_h, int64_t d_c,
+                               const gmla_bf16 *W_k, const gmla_bf16 *W_v, float scale,
+                               const gmla_bf16 *G, gmla_bf16 *O, float *weights, void *workspace,
+                               size_t workspace_bytes, gmla_stream_t stream);
+GMLA_API size_t gmla_attend_decode_workspace_size(int64_t B, int64_t L, int64_t H, int64_t d_c);
+
+/*
+ * gmla_gate_out -- the output projection Y = O W_o^T over M = B*T rows.
+ * "Gated MLA" page, "The channel-wise output gate" (gate before W_o) and
+ * step 6.  The gate is applied upstream (gmla_attend_prefill and
+ * gmla_attend_decode take G); passing G != NULL here returns
+ * GMLA_ERR_UNSUPPORTED.
+ *
+ *  O [M, d_model] gated context; W_o [d_model, d_model]; Y [M, d_model].
+ *  workspace >= gmla_gate_out_workspace_size(M, d_model) bytes.
+ */
+GMLA_API gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M,
+                          int64_t d_model, gmla_bf16 *Y, void *workspace, size_t workspace_bytes,
+                          gmla_stream_t stream);
+GMLA_API size_t gmla_gate_out_workspace_size(int64_t M, int64_t d_model);
+
+/* Synchronise `stream`, then read and clear this device's status word.
+ * Returns GMLA_OK, GMLA_ERR_TIMEOUT (a bounded wait ran out) or GMLA_ERR_CUDA. */
+GMLA_API gmla_status gmla_get_device_status(gmla_stream_t stream);
+
+/* Static, NUL-terminated description of a status code (host memory, never freed). */
+GMLA_API const char *gmla_status_string(gmla_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+GMLA_API int gmla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GMLA_H */

@@ -1,0 +1,101 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol that
+include/gmla.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "gmla.h")
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"GMLA_API\s+[\w\s\*]+?\b(gmla_\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def gmla():
+    from causal_head_latent_b200 import build
+    build.build()
+    import causal_head_latent_b200 as g
+    return g
+
+
+def test_header_declares_the_four_calls():
+    syms = declared_symbols()
+    for name in ("gmla_latent_project", "gmla_attend_prefill", "gmla_attend_decode", "gmla_gate_out"):
+        assert name in syms
+    assert len(syms) >= 10
+
+
+def test_library_exports_every_declared_symbol(gmla):
+    out = subprocess.run(["nm", "-D", "--defined-only", gmla.library_path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (gmla_\w+)", out))
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(gmla.lib, name)
+    # nothing else leaks from the library's C++ internals
+    assert not [s for s in re.findall(r"\bT (\S+)", out) if "gmla" in s and not s.startswith("gmla_")]
+
+
+def test_status_strings_and_version(gmla):
+    for code in range(6):
+        assert gmla.gmla_status_string(code)
+    assert gmla.gmla_version() >= 100
+
+
+def _i3(*v):
+    return (ctypes.c_int64 * 3)(*v)
+
+
+def test_host_validation_without_gpu(gmla):
+    L = gmla.lib
+    fake = 0x10000  # never dereferenced: every call below fails validation first
+    s = _i3(128 * 2 * 300, 128 * 2, 128)
+    # null Q
+    assert L.gmla_attend_prefill(None, s, fake, s, fake, s, 1, 2, 300, 300, 128, 1, 0.0, None, fake, s, None, None,
+                                 None) == 1
+    # Tq > Tk
+    assert L.gmla_attend_prefill(fake, s, fake, s, fake, s, 1, 2, 301, 300, 128, 1, 0.0, None, fake, s, None, None,
+                                 None) == 1
+    # causal flag not boolean
+    assert L.gmla_attend_prefill(fake, s, fake, s, fake, s, 1, 2, 300, 300, 128, 2, 0.0, None, fake, s, None, None,
+                                 None) == 1
+    # misaligned pointer
+    assert L.gmla_attend_prefill(fake + 2, s, fake, s, fake, s, 1, 2, 300, 300, 128, 1, 0.0, None, fake, s, None,
+                                 None, None) == 1
+    # stride not a multiple of 8 elements
+    assert L.gmla_attend_prefill(fake, _i3(100, 12, 4), fake, s, fake, s, 1, 2, 300, 300, 128, 1, 0.0, None, fake, s,
+                                 None, None, None) == 1
+    # head width other than 128
+    assert L.gmla_attend_prefill(fake, s, fake, s, fake, s, 1, 2, 300, 300, 64, 1, 0.0, None, fake, s, None, None,
+                                 None) == 2
+    # latent project: cache too short, K requested without C, d_model not a multiple of 128
+    assert L.gmla_latent_project(fake, 2, 10, 256, fake, fake, fake, 64, fake, fake, fake, fake, fake, 15, 6, None,
+                                 None, None, 0, None) == 1
+    assert L.gmla_latent_project(fake, 2, 10, 256, fake, fake, fake, 64, fake, fake, fake, fake, None, 16, 0, fake,
+                                 None, None, 0, None) == 1
+    assert L.gmla_latent_project(fake, 2, 10, 200, fake, fake, fake, 64, fake, fake, fake, fake, fake, 16, 0, None,
+                                 None, None, 0, None) == 2
+    # decode: L beyond the cache, and a short workspace
+    assert L.gmla_attend_decode(fake, fake, 2, 100, 101, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 1 << 30,
+                                None) == 1
+    assert L.gmla_attend_decode(fake, fake, 2, 100, 100, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 16,
+                                None) == 5
+    assert L.gmla_attend_decode_workspace_size(2, 100, 2, 64) > 16
+    # gate_out: the gate is fused upstream
+    assert L.gmla_gate_out(fake, fake, fake, 4, 256, fake, None, 0, None) == 2
+    assert L.gmla_gate_out(None, None, fake, 4, 256, fake, None, 0, None) == 1
+
+
+def test_binding_has_no_cpu_path():
+    import causal_head_latent_b200 as g
+    src = open(os.path.join(ROOT, "causal_head_latent_b200", "__init__.py")).read()
+    assert "oracle" not in src and "numpy" not in src
+    assert callable(g.gmla_attend_prefill)

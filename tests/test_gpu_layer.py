@@ -1,0 +1,128 @@
+"""GPU parity: projections (gmla_latent_project), output projection
+(gmla_gate_out), latent-cache decode (gmla_attend_decode) and the chained
+layer, against the float64 oracle through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from synth_inputs import SEEDS, Draw, layer_weights
+from tests.gpu_util import ROW_SUM, assert_parity, bits, f64, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    import causal_head_latent_b200 as gm
+    return gm
+
+
+def make_layer(seed, B, T, d, d_c):
+    dr = Draw(seed)
+    w = layer_weights(dr, d, d_c, x_shape=(B, T, d))
+    return w, {k: to_dev(v) for k, v in w.items()}
+
+
+def ws(nbytes):
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("B,T,d,d_c,cache_len_max,cache_pos", [(2, 200, 256, 64, 200, 0), (1, 130, 384, 128, 300, 17),
+                                                               (3, 1, 256, 64, 9, 8)])
+def test_latent_project_matches_oracle(g, B, T, d, d_c, cache_len_max, cache_pos):
+    w, t = make_layer(200 + T, B, T, d, d_c)
+    Q = torch.empty(B, T, d, dtype=torch.bfloat16, device="cuda")
+    G = torch.empty_like(Q)
+    K = torch.empty_like(Q)
+    V = torch.empty_like(Q)
+    C = torch.zeros(B, cache_len_max, d_c, dtype=torch.bfloat16, device="cuda")
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=Q, G=G, C=C,
+                          cache_pos=cache_pos, K=K, V=V)
+    g.gmla_get_device_status()
+    assert_parity(f64(Q), orc.linear(w["X"], w["W_q"]), "Q")
+    assert_parity(f64(G), orc.linear(w["X"], w["W_g"]), "G")
+    Cg = f64(C)
+    assert_parity(Cg[:, cache_pos:cache_pos + T], orc.linear(w["X"], w["W_c"]), "C")
+    # rows outside [cache_pos, cache_pos + T) untouched
+    assert np.all(Cg[:, :cache_pos] == 0) and np.all(Cg[:, cache_pos + T:] == 0)
+    # K, V are expanded from the latents as stored in bfloat16; the oracle rounds its
+    # own latents at the same boundary (no GPU value feeds the oracle)
+    Cr = orc.round_bf16(orc.linear(w["X"], w["W_c"]))
+    assert_parity(f64(K), orc.linear(Cr, w["W_k"]), "K")
+    assert_parity(f64(V), orc.linear(Cr, w["W_v"]), "V")
+
+
+def test_gate_out_matches_oracle(g):
+    rng = np.random.default_rng(3)
+    from synth_inputs import bf16_bits_from_f64
+    M, d = 300, 384
+    O = bf16_bits_from_f64(rng.standard_normal((M, d)))
+    W = bf16_bits_from_f64(rng.standard_normal((d, d)) / np.sqrt(d))
+    Y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    g.gmla_gate_out(to_dev(O), to_dev(W), Y)
+    g.gmla_get_device_status()
+    assert_parity(f64(Y), orc.linear(O, W), "Y")
+
+
+def test_layer_chained_matches_oracle(g):
+    """X -> projections -> attention (+ gate) -> W_o, against the oracle that rounds
+    to bfloat16 at the same library boundaries."""
+    B, T, H, d_c = 2, 300, 3, 128
+    d = 128 * H
+    w, t = make_layer(17, B, T, d, d_c)
+    Q = torch.empty(B, T, d, dtype=torch.bfloat16, device="cuda")
+    G, K, V, O, Y = (torch.empty_like(Q) for _ in range(5))
+    C = torch.empty(B, T, d_c, dtype=torch.bfloat16, device="cuda")
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=Q, G=G, C=C, K=K, V=V)
+    g.gmla_attend_prefill(Q.view(B, T, H, 128), K.view(B, T, H, 128), V.view(B, T, H, 128), O.view(B, T, H, 128),
+                          G=G)
+    g.gmla_gate_out(O, t["W_o"], Y)
+    g.gmla_get_device_status()
+    ref = orc.gated_mla(w["X"], w["W_q"], w["W_c"], w["W_k"], w["W_v"], w["W_g"], w["W_o"], H,
+                        round_boundaries=True, intermediates=True)
+    assert_parity(f64(C), ref["latent_cache"], "latent cache")
+    assert_parity(f64(O), ref["O_gated"], "gated context")
+    assert_parity(f64(Y), ref["output"], "Y")
+    assert Y.shape == t["X"].shape and Y.dtype == t["X"].dtype
+
+
+@pytest.mark.parametrize("B,L,Lmax,H,d_c", [(3, 700, 700, 4, 128), (2, 1, 5, 2, 64), (1, 2049, 3000, 3, 512)])
+def test_attend_decode_matches_oracle(g, B, L, Lmax, H, d_c):
+    d = 128 * H
+    dr = Draw(300 + L)
+    q = dr.normal((B, d))
+    cache = dr.normal((B, Lmax, d_c))
+    Wk = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Wv = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Gl = dr.normal((B, d))
+    O = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    W = torch.full((B, H, L), float("nan"), device="cuda")
+    work = ws(g.gmla_attend_decode_workspace_size(B, L, H, d_c))
+    g.gmla_attend_decode(to_dev(q), to_dev(cache), L, to_dev(Wk), to_dev(Wv), O, H, G=to_dev(Gl), weights=W,
+                         workspace=work)
+    g.gmla_get_device_status()
+    ref, wref = orc.decode_latent(q, cache, L, Wk, Wv, H, G=Gl, want_weights=True)
+    assert_parity(f64(O), ref, "decode O")
+    w = f64(W)
+    assert np.abs(w.sum(-1) - 1.0).max() <= ROW_SUM
+    assert np.abs(w - wref).max() < 1e-4
+
+
+def test_decode_equals_prefill_last_row(g):
+    """Decode of token t over latents 0..t equals row t of causal prefill (same GPU inputs)."""
+    B, T, H, d_c = 1, 257, 2, 128
+    d = 128 * H
+    w, t = make_layer(23, B, T, d, d_c)
+    Q = torch.empty(B, T, d, dtype=torch.bfloat16, device="cuda")
+    G, K, V, O = (torch.empty_like(Q) for _ in range(4))
+    C = torch.empty(B, T, d_c, dtype=torch.bfloat16, device="cuda")
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=Q, G=G, C=C, K=K, V=V)
+    g.gmla_attend_prefill(Q.view(B, T, H, 128), K.view(B, T, H, 128), V.view(B, T, H, 128), O.view(B, T, H, 128),
+                          G=G)
+    Od = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    work = ws(g.gmla_attend_decode_workspace_size(B, T, H, d_c))
+    g.gmla_attend_decode(Q[:, -1].contiguous(), C, T, t["W_k"], t["W_v"], Od, H, G=G[:, -1].contiguous(),
+                         workspace=work)
+    g.gmla_get_device_status()
+    assert_parity(f64(Od), f64(O[:, -1]), "decode vs prefill row", rel_l2=1e-2)
