@@ -1,0 +1,554 @@
+"""Benchmark of the Gated MLA hot path on B200.
+
+One step = one pass of the hot path over one synthetic batch:
+  prefill  causal attention, B=1, 96 heads, T=8192, D_h=128 (gmla_attend_prefill)
+  decode   one new token for B=32 sequences over L=131072 cached latents of width
+           512: projections of the new token with the latent appended at row
+           L-1 (gmla_latent_project), absorbed attention over the latent cache
+           with log-sum-exp combine and gate (gmla_attend_decode), W_o
+           (gmla_gate_out); d_model = 12288.
+Headline value: prefill attention TFLOP/s (causal pairs only:
+4*D_h*H*B*T(T+1)/2 flop).  The decode half of the metric -- latent-cache GB/s
+of gmla_attend_decode -- is reported in the "decode" object.  Both inputs are
+larger than L2 (Q/K/V 604 MB, cache 4.3 GB), so no flush is needed between
+steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--parts all|prefill|decode] [--workload step|layer]
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs the same
+per-GPU workload (data-parallel replicas, no collective on the data path);
+value is the total over ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attention TFLOP/s & decode latent-cache GB/s, % of B200 roofline"
+
+# workload sizes
+P_B, P_H, P_T, D = 1, 96, 8192, 128
+DEC_B, DEC_L, DC, DM = 32, 131072, 512, 12288
+L_B, L_T = 2, 4096   # --workload layer: full layer prefill
+
+
+def prefill_flops(B=P_B, H=P_H, T=P_T):
+    return 4.0 * D * H * B * T * (T + 1) / 2
+
+
+def decode_bytes(B=DEC_B, L=DEC_L, H=96, dc=DC):
+    # algorithmic bytes of gmla_attend_decode: the visible latents, W_k, W_v, q, G and O
+    d = H * D
+    return 2.0 * (B * L * dc + 2 * d * dc + 3 * B * d)
+
+
+def decode_step_bytes(B=DEC_B, L=DEC_L, dc=DC, dm=DM):
+    # whole decode step: attend_decode plus W_q, W_g, W_c, W_o and the new-token activations
+    return decode_bytes(B, L, dm // D, dc) + 2.0 * (3 * dm * dm + dc * dm + 4 * B * dm + B * dc)
+
+
+def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
+    M = B * T
+    return 2.0 * M * d * (2 * d + dc) + 2.0 * M * dc * 2 * d + prefill_flops(B, d // D, T) + 2.0 * M * d * d
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n_gpus > 1 and world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} needs torch.distributed.run with {n_gpus} processes (WORLD_SIZE={world})")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workloads
+
+
+def dev(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+class PrefillPart:
+    """Causal prefill attention B=1, H=96, T=8192."""
+
+    def __init__(self, seed):
+        import torch
+        from synth_inputs import prefill_qkv
+        inp = prefill_qkv(seed, P_B, P_T, P_H)
+        self.host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in inp.items()}
+        self.Q, self.K, self.V = (self.host[k].cuda() for k in ("Q", "K", "V"))
+        self.O = torch.empty_like(self.Q)
+        self.O_host = torch.empty(self.O.shape, dtype=torch.bfloat16).pin_memory()
+        self.flops = prefill_flops()
+        self.launches = 1
+
+    def run(self):
+        import causal_head_latent_b200 as g
+        g.gmla_attend_prefill(self.Q, self.K, self.V, self.O, causal=True)
+
+    def run_e2e(self):
+        """Through the public API with host buffers: H2D of Q, K, V, the call, D2H of O."""
+        import causal_head_latent_b200 as g
+        for k, t in (("Q", self.Q), ("K", self.K), ("V", self.V)):
+            t.copy_(self.host[k], non_blocking=True)
+        g.gmla_attend_prefill(self.Q, self.K, self.V, self.O, causal=True)
+        self.O_host.copy_(self.O, non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = sum(self.host[k].numel() * 2 for k in ("Q", "K", "V"))
+        return h2d, self.O.numel() * 2
+
+
+class DecodePart:
+    """One decode step: B=32 new tokens over L=131072 cached latents (d_c=512), d_model=12288."""
+
+    def __init__(self, seed):
+        import torch
+
+        import causal_head_latent_b200 as g
+        from synth_inputs import Draw, layer_weights
+        dr = Draw(seed)
+        w = layer_weights(dr, DM, DC, x_shape=(DEC_B, 1, DM))
+        cache = dr.normal((DEC_B, DEC_L, DC))
+        self.W = {k: dev(v) for k, v in w.items() if k != "X"}
+        self.X_host = torch.from_numpy(w["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.X = self.X_host.cuda()
+        self.C = dev(cache)
+        del cache
+        self.Q = torch.empty(DEC_B, 1, DM, dtype=torch.bfloat16, device="cuda")
+        self.G = torch.empty_like(self.Q)
+        self.O = torch.empty(DEC_B, DM, dtype=torch.bfloat16, device="cuda")
+        self.Y = torch.empty_like(self.O)
+        self.Y_host = torch.empty(self.Y.shape, dtype=torch.bfloat16).pin_memory()
+        self.ws_p = torch.empty(max(1, g.gmla_latent_project_workspace_size(DEC_B, 1, DM, DC)), dtype=torch.uint8,
+                                device="cuda")
+        self.ws_d = torch.empty(g.gmla_attend_decode_workspace_size(DEC_B, DEC_L, DM // D, DC), dtype=torch.uint8,
+                                device="cuda")
+        self.ws_o = torch.empty(max(1, g.gmla_gate_out_workspace_size(DEC_B, DM)), dtype=torch.uint8, device="cuda")
+        self.bytes = decode_bytes()
+        self.launches = 6
+
+    def project(self):
+        import causal_head_latent_b200 as g
+        W = self.W
+        g.gmla_latent_project(self.X, W["W_q"], W["W_g"], W["W_c"], None, None, Q=self.Q, G=self.G, C=self.C,
+                              cache_pos=DEC_L - 1, workspace=self.ws_p)
+
+    def attend(self):
+        import causal_head_latent_b200 as g
+        g.gmla_attend_decode(self.Q.view(DEC_B, DM), self.C, DEC_L, self.W["W_k"], self.W["W_v"], self.O, DM // D,
+                             G=self.G.view(DEC_B, DM), workspace=self.ws_d)
+
+    def out(self):
+        import causal_head_latent_b200 as g
+        g.gmla_gate_out(self.O, self.W["W_o"], self.Y, workspace=self.ws_o)
+
+    def run_e2e(self):
+        self.X.copy_(self.X_host, non_blocking=True)
+        self.project()
+        self.attend()
+        self.out()
+        self.Y_host.copy_(self.Y, non_blocking=True)
+
+
+class LayerPart:
+    """Full Gated MLA layer prefill: B=2, T=4096, d_model=12288, d_c=512."""
+
+    def __init__(self, seed):
+        import torch
+        from synth_inputs import Draw, layer_weights
+        w = layer_weights(Draw(seed), DM, DC, x_shape=(L_B, L_T, DM))
+        self.t = {k: dev(v) for k, v in w.items()}
+        self.Q = torch.empty(L_B, L_T, DM, dtype=torch.bfloat16, device="cuda")
+        self.G, self.K, self.V, self.O, self.Y = (torch.empty_like(self.Q) for _ in range(5))
+        self.C = torch.empty(L_B, L_T, DC, dtype=torch.bfloat16, device="cuda")
+        self.flops = layer_flops()
+        self.launches = 4
+
+    def run(self):
+        import causal_head_latent_b200 as g
+        t = self.t
+        H = DM // D
+        g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=self.Q, G=self.G, C=self.C,
+                              K=self.K, V=self.V)
+        v = lambda x: x.view(L_B, L_T, H, D)
+        g.gmla_attend_prefill(v(self.Q), v(self.K), v(self.V), v(self.O), G=self.G)
+        g.gmla_gate_out(self.O, t["W_o"], self.Y)
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+
+
+def oracle_prefill_sample(seconds_target=15.0, rows=None, inp=None):
+    """Time the float64 oracle on a bounded sample of the prefill workload: `rows`
+    query rows (b=0, random head and position) of the B=1, H=96, T=8192 problem."""
+    import oracle as orc
+    from synth_inputs import SEEDS, prefill_qkv
+    if inp is None:
+        # widened to float64 once, outside the timed call
+        inp = {k: orc.widen(v) for k, v in prefill_qkv(SEEDS["prefill_attn"], P_B, P_T, P_H).items()}
+    rng = np.random.default_rng(1)
+    if rows is None:
+        rows = 2000
+    sel = np.stack([np.zeros(rows, np.int64), rng.integers(0, P_H, rows), rng.integers(0, P_T, rows)], 1)
+    flops = float(np.sum(4.0 * D * (sel[:, 2] + 1)))
+    t0 = time.perf_counter()
+    orc.attention(inp["Q"], inp["K"], inp["V"], rows=sel)
+    dt = time.perf_counter() - t0
+    return flops, dt, rows, orc.num_threads(), inp
+
+
+def cpu_baseline_prefill(target_s=15.0):
+    flops, dt, rows, cores, inp = oracle_prefill_sample(rows=500)
+    n = int(max(500, min(200000, 500 * target_s / max(dt, 1e-3))))
+    flops, dt, rows, cores, _ = oracle_prefill_sample(rows=n, inp=inp)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} random query rows (b=0, random head, random position) of the B=1 H=96 T=8192 causal "
+                      f"prefill, float64 C oracle, {dt:.1f} s"}
+
+
+def cpu_baseline_decode(target_s=8.0):
+    """Oracle decode (plain definition: K_h, V_h rebuilt from the cache) for a few
+    (b, h) pairs over the first `L` latents; GB/s counts the cache bytes a full
+    decode step would stream at the same per-(b,h) rate."""
+    import oracle as orc
+    from synth_inputs import Draw
+    dr = Draw(77)
+    L = 8192
+    H = 96
+    q = dr.normal((1, DM))
+    cache = dr.normal((1, L, DC))
+    Wk = dr.normal((DM, DC), 1 / math.sqrt(DC))
+    Wv = dr.normal((DM, DC), 1 / math.sqrt(DC))
+    heads = [(0, h) for h in range(0, H, 12)]
+    t0 = time.perf_counter()
+    orc.decode_latent(q, cache, L, Wk, Wv, H, heads=heads)
+    dt = time.perf_counter() - t0
+    # full step = DEC_B * H (b, h) pairs over DEC_L latents; per-(b,h) time scales with L
+    t_full = dt / len(heads) * (DEC_B * H) * (DEC_L / L)
+    return {"value": decode_bytes() / t_full / 1e9, "unit": "GB/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{len(heads)} (b,h) pairs over L={L} latents (non-absorbed float64 C oracle, {dt:.1f} s), "
+                      f"scaled to B=32 x 96 heads x L=131072"}
+
+
+# ------------------------------------------------------------------ main
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the float64 oracle timed on the host cores."""
+    if rank != 0:
+        return
+    flops0, dt0, _, cores, inp = oracle_prefill_sample(rows=200)
+    rows = int(max(200, min(20000, 200 * 2.0 / max(dt0, 1e-3))))   # about 2 s per step
+    for _ in range(args.warmup):
+        oracle_prefill_sample(rows=rows, inp=inp)
+    tot_f = tot_t = 0.0
+    for _ in range(args.steps):
+        f, dt, _, cores, _ = oracle_prefill_sample(rows=rows, inp=inp)
+        tot_f += f
+        tot_t += dt
+    val = tot_f / tot_t / 1e12
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_obj(args),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"per step {rows} random query rows of the B=1 H=96 T=8192 causal prefill"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_obj(args):
+    if args.workload == "layer":
+        return {"workload": f"Gated MLA layer prefill B={L_B} T={L_T} d_model={DM} H=96 D_h=128 d_c={DC} bf16",
+                "global_batch": L_B * max(1, args.gpus), "seq_len": L_T, "parallelism": f"dp{args.gpus}",
+                "l2": "inputs larger than L2"}
+    return {"workload": f"causal prefill attention B={P_B} H={P_H} T={P_T} D_h={D} bf16 + latent-cache decode "
+                        f"B={DEC_B} L={DEC_L} d_c={DC} H=96 d_model={DM} (projections, append, absorbed attention, "
+                        f"LSE combine, gate, W_o)",
+            "global_batch": P_B * max(1, args.gpus), "seq_len": P_T, "parallelism": f"dp{args.gpus}",
+            "parts": args.parts, "l2": "inputs larger than L2 (Q/K/V 604 MB, cache 4.3 GB); no flush"}
+
+
+def timed(fn_list, steps, world):
+    """Run `steps` iterations of every fn in fn_list; per-fn CUDA-event time on the
+    current stream; the whole region bracketed by barrier + synchronize."""
+    import torch
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in fn_list]
+          for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    start.record()
+    for i in range(steps):
+        for j, fn in enumerate(fn_list):
+            ev[i][j][0].record()
+            fn()
+            ev[i][j][1].record()
+    end.record()
+    barrier(world)
+    total = start.elapsed_time(end)
+    per = [sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)) for j in range(len(fn_list))]
+    return total, per
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--parts", default="all", choices=["all", "prefill", "decode"])
+    ap.add_argument("--workload", default="step", choices=["step", "layer"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+
+    import torch
+    rank, world, local = dist_setup(args.gpus)
+    import causal_head_latent_b200 as g
+    peaks = load_peaks()
+
+    if args.workload == "layer":
+        part = LayerPart(4)
+        for _ in range(args.warmup):
+            part.run()
+        g.gmla_get_device_status()
+        clk = ClockSampler(local)
+        clk.start()
+        total, per = timed([part.run], args.steps, world)
+        clocks = clk.stop()
+        g.gmla_get_device_status()
+        total = max_over_ranks(total, world)
+        val = part.flops * args.steps * world / (total / 1e3) / 1e12
+        line = {"metric": "Gated MLA layer prefill TFLOP/s", "value": val, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": config_obj(args), "clocks": clocks,
+                "gpu_launches": part.launches * args.steps,
+                "roofline": {"bound": "tensor", "achieved": val / world,
+                             "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                             "frac": val / world / peaks["bf16_tflops_sustained"], "traffic": None,
+                             "peak_kind": f"{peaks['source']} sustained bf16"}}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
+
+    parts = []
+    pre = dec = None
+    if args.parts in ("all", "prefill"):
+        pre = PrefillPart(3)
+    if args.parts in ("all", "decode"):
+        dec = DecodePart(5)
+    fns, names = [], []
+    if pre:
+        fns.append(pre.run)
+        names.append("prefill_attention")
+    if dec:
+        fns += [dec.project, dec.attend, dec.out]
+        names += ["decode_project", "decode_attend", "decode_out"]
+
+    for _ in range(args.warmup):
+        for fn in fns:
+            fn()
+    g.gmla_get_device_status()
+
+    clk = ClockSampler(local)
+    clk.start()
+    total, per = timed(fns, args.steps, world)
+    clocks = clk.stop()
+    g.gmla_get_device_status()
+    total = max_over_ranks(total, world)
+    per = [max_over_ranks(p, world) for p in per]
+    perd = dict(zip(names, per))
+    K = args.steps
+    launches = (1 if pre else 0) + (dec.launches if dec else 0)
+
+    line = {"metric": METRIC, "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_obj(args), "clocks": clocks, "gpu_launches": launches * K,
+            "kernel_ms_per_step": {k: v / K for k, v in perd.items()}}
+    if pre:
+        t_att = perd["prefill_attention"] / K
+        val = pre.flops * world / (t_att / 1e3) / 1e12
+        line.update(value=val, unit="TFLOP/s")
+        ach = pre.flops / (t_att / 1e3) / 1e12
+        line["roofline"] = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
+                            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                            "kernel": "attn_prefill_kernel",
+                            "peak_kind": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)",
+                            "frac_of_burst": ach / peaks["bf16_tflops"], "frac_of_datasheet_2250": ach / 2250.0}
+    if dec:
+        t_dec = perd["decode_attend"] / K
+        gbs = dec.bytes / (t_dec / 1e3) / 1e9
+        t_step = (perd["decode_project"] + perd["decode_attend"] + perd["decode_out"]) / K
+        dobj = {"value": gbs * world, "unit": "GB/s", "ms_per_step": t_dec,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "gmla_attend_decode",
+                             "peak_kind": f"{peaks['source']} HBM copy", "frac_of_datasheet_8000": gbs / 8000.0},
+                "step_ms": t_step, "step_gbs": decode_step_bytes() / (t_step / 1e3) / 1e9}
+        line["decode"] = dobj
+        if not pre:
+            line.update(value=gbs * world, unit="GB/s", roofline=dobj["roofline"])
+
+    # end-to-end through the public API with pinned host buffers
+    if not args.no_e2e:
+        ke = max(1, min(K, 5))
+        if pre:
+            for _ in range(1):
+                pre.run_e2e()
+            barrier(world)
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(ke):
+                pre.run_e2e()
+            t1.record()
+            barrier(world)
+            te = max_over_ranks(t0.elapsed_time(t1), world) / ke
+            h2d, d2h = pre.e2e_bytes()
+            line["e2e"] = {"value": pre.flops * world / (te / 1e3) / 1e12, "unit": "TFLOP/s",
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": te,
+                           "what": "H2D of Q, K, V from pinned host memory + gmla_attend_prefill + D2H of O"}
+        if dec:
+            dec.run_e2e()
+            barrier(world)
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(ke):
+                dec.run_e2e()
+            t1.record()
+            barrier(world)
+            te = max_over_ranks(t0.elapsed_time(t1), world) / ke
+            e = {"value": dec.bytes * world / (te / 1e3) / 1e9, "unit": "GB/s",
+                 "h2d_bytes_per_step": dec.X_host.numel() * 2, "d2h_bytes_per_step": dec.Y_host.numel() * 2,
+                 "ms_per_step": te, "what": "H2D of the new tokens' hidden states + full decode step "
+                                            "(projections, append, attend, W_o) + D2H of Y; cache and weights resident"}
+            line["decode"]["e2e"] = e
+            if not pre:
+                line["e2e"] = e
+        g.gmla_get_device_status()
+
+    if rank == 0 and world >= 1 and not args.no_cpu:
+        if pre:
+            line["cpu_baseline"] = cpu_baseline_prefill()
+        if dec:
+            cb = cpu_baseline_decode()
+            line["decode"]["cpu_baseline"] = cb
+            if not pre:
+                line["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
