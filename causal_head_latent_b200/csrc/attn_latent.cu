@@ -5,25 +5,31 @@
 // latents c_0..c_{L-1} ("Gated MLA" page: K = C W_k^T, V = C W_v^T), the
 // head-h scores are q_h . (W_k^(h) c_s) = (W_k^(h)T q_h) . c_s and the head
 // context is sum_s a_s W_v^(h) c_s = W_v^(h) (sum_s a_s c_s), with W^(h) the
-// rows h*D .. h*D+D-1.  Three steps:
-//   absorb   q~[b,h,:] = scale * log2(e) * W_k^(h)T q_h          (float32)
-//   stream   per key split: running max m, sum l and acc[h,:] = sum_s p_s c_s
-//            over the latents, every latent read once for all heads
+// rows h*D .. h*D+D-1.  Three launches:
+//   absorb   q~[b,h,:] = scale * log2(e) * W_k^(h)T q_h, stored as bfloat16
+//   stream   tensor-core split-KV pass over the latents (attn_latent_tc.cu):
+//            per split the running max m, sum l and acc[h,:] = sum_s p_s c_s
 //   combine  exact log-sum-exp merge of the splits, c^ = acc / l, then
-//            o_h = W_v^(h) c^_h, gate sigmoid(G), bf16 store.
+//            o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store.
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace gmla {
+
+int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, int B, int L, int H, int dc, int n_splits,
+                     int keys_per_split, float *part_m, float *part_l, float *part_acc, float *weights,
+                     unsigned *status, cudaStream_t stream);
+int latent_tc_tile_keys();
+
 namespace latent {
 
 constexpr int HD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- absorb
-// grid (H, d_c / 128), 128 threads: thread j owns latent column c = 128*y + j.
+// grid (H, ceil(d_c / 128)), 128 threads: thread j owns latent column c = 128*y + j.
 __global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ Wk,
-                                                     int B, int H, int dc, float sl2, float *__restrict__ qt) {
+                                                     int B, int H, int dc, float sl2, uint16_t *__restrict__ qt) {
   extern __shared__ float qs[];  // [B][HD]
   const int h = blockIdx.x;
   const int c = blockIdx.y * 128 + threadIdx.x;
@@ -46,155 +52,78 @@ __global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict_
     }
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (j < nb) qt[((size_t)(b0 + j) * H + h) * dc + c] = acc[j] * sl2;
-  }
-}
-
-// ---------------------------------------------------------------- stream (CUDA-core version)
-// grid (n_splits, H / HG, B), 256 threads; HG heads per CTA, KT keys per tile.
-constexpr int HG = 8;
-constexpr int KT = 32;
-constexpr int ST = 256;
-
-struct StreamParams {
-  const uint16_t *C;
-  long long cache_len_max;
-  int L, H, dc, n_splits, keys_per_split;
-  const float *qt;       // [B,H,dc]
-  float *part_m, *part_l, *part_acc;  // [S,B,H], [S,B,H], [S,B,H,dc]
-  float *weights;        // optional raw scores [B,H,L]
-  int B;
-};
-
-__global__ void __launch_bounds__(ST) stream_kernel(const StreamParams P) {
-  extern __shared__ float sm[];
-  const int dc = P.dc;
-  float *q_s = sm;                 // [HG][dc]
-  float *c_s = q_s + HG * dc;      // [KT][dc]
-  float *p_s = c_s + KT * dc;      // [HG][KT]
-  float *m_s = p_s + HG * KT;      // [HG]
-  float *a_s = m_s + HG;           // [HG] rescale factors
-  const int split = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-  const int h0 = hg * HG;
-  const int k_begin = split * P.keys_per_split;
-  const int k_end = min(P.L, k_begin + P.keys_per_split);
-  for (int i = threadIdx.x; i < HG * dc; i += ST) {
-    const int hh = i / dc, c = i % dc;
-    q_s[i] = (h0 + hh < P.H) ? P.qt[((size_t)b * P.H + h0 + hh) * dc + c] : 0.f;
-  }
-  // each thread owns outputs (head hh, column c) for idx = tid + ST*j
-  const int per = (HG * dc) / ST;  // dc multiple of 64 -> per = dc/32
-  float acc[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;  // meaningful in threads < HG
-  if (threadIdx.x < HG) m_s[threadIdx.x] = -INFINITY;
-  __syncthreads();
-  for (int k0 = k_begin; k0 < k_end; k0 += KT) {
-    const int nk = min(KT, k_end - k0);
-    for (int i = threadIdx.x; i < KT * dc; i += ST) {
-      const int kk = i / dc, c = i % dc;
-      c_s[i] = kk < nk ? bf16_to_f32(P.C[((size_t)b * P.cache_len_max + k0 + kk) * dc + c]) : 0.f;
-    }
-    __syncthreads();
-    // scores: thread -> (head, key)
-    {
-      const int hh = threadIdx.x / KT, kk = threadIdx.x % KT;
-      float s = -INFINITY;
-      if (kk < nk) {
-        float d = 0.f;
-        for (int c = 0; c < dc; ++c) d = fmaf(q_s[hh * dc + c], c_s[kk * dc + c], d);
-        s = d;
-        if (P.weights && h0 + hh < P.H) P.weights[((size_t)b * P.H + h0 + hh) * P.L + k0 + kk] = s;
-      }
-      p_s[hh * KT + kk] = s;
-    }
-    __syncthreads();
-    if (threadIdx.x < HG) {
-      const int hh = threadIdx.x;
-      float mx = m_run;
-      for (int kk = 0; kk < nk; ++kk) mx = fmaxf(mx, p_s[hh * KT + kk]);
-      const float alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - mx);
-      float ls = 0.f;
-      for (int kk = 0; kk < KT; ++kk) {
-        const float pv = kk < nk ? fast_exp2(p_s[hh * KT + kk] - mx) : 0.f;
-        ls += pv;
-        p_s[hh * KT + kk] = __bfloat162float(__float2bfloat16_rn(pv));
-      }
-      l_run = l_run * alpha + ls;
-      m_run = mx;
-      a_s[hh] = alpha;
-    }
-    __syncthreads();
-    for (int j = 0; j < per; ++j) {
-      const int idx = threadIdx.x + ST * j;
-      const int hh = idx / dc, c = idx % dc;
-      float a = acc[j] * a_s[hh];
-      for (int kk = 0; kk < nk; ++kk) a = fmaf(p_s[hh * KT + kk], c_s[kk * dc + c], a);
-      acc[j] = a;
-    }
-    __syncthreads();
-  }
-  const size_t base = ((size_t)split * P.B + b) * P.H;
-  if (threadIdx.x < HG && h0 + threadIdx.x < P.H) {
-    P.part_m[base + h0 + threadIdx.x] = m_run;
-    P.part_l[base + h0 + threadIdx.x] = l_run;
-  }
-  for (int j = 0; j < per; ++j) {
-    const int idx = threadIdx.x + ST * j;
-    const int hh = idx / dc, c = idx % dc;
-    if (h0 + hh < P.H) P.part_acc[(base + h0 + hh) * dc + c] = acc[j];
+      if (j < nb) qt[((size_t)(b0 + j) * H + h) * dc + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j] * sl2));
   }
 }
 
 // ---------------------------------------------------------------- combine + W_v + gate
-// grid (H, B), 128 threads (one per output channel of the head).
+// grid (H, ceil(B / CB)), 128 threads (one per output channel of the head).
+constexpr int CB = 8;
+
 struct CombineParams {
   const float *part_m, *part_l, *part_acc;
   int n_splits, B, H, dc;
   const uint16_t *Wv, *G;
   uint16_t *O;
-  float *lse2;  // [B,H] log2-domain lse (for debug weights)
+  float *lse2;  // [B,H] log2-domain log-sum-exp (for the debug weights)
 };
 
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams P) {
-  extern __shared__ float chat[];  // [dc]
-  const int h = blockIdx.x, b = blockIdx.y;
+  extern __shared__ float chat[];  // [CB][dc]
+  const int h = blockIdx.x, b0 = blockIdx.y * CB;
+  const int nb = min(CB, P.B - b0);
   const int dc = P.dc;
-  float M = -INFINITY;
-  for (int s = 0; s < P.n_splits; ++s) M = fmaxf(M, P.part_m[((size_t)s * P.B + b) * P.H + h]);
-  float Lsum = 0.f;
-  for (int s = 0; s < P.n_splits; ++s) {
-    const float ms = P.part_m[((size_t)s * P.B + b) * P.H + h];
-    if (ms != -INFINITY) Lsum += P.part_l[((size_t)s * P.B + b) * P.H + h] * fast_exp2(ms - M);
-  }
-  const float inv = 1.f / Lsum;
-  for (int c = threadIdx.x; c < dc; c += 128) {
-    float a = 0.f;
+  for (int bb = 0; bb < nb; ++bb) {
+    const int b = b0 + bb;
+    float M = -INFINITY;
+    for (int s = 0; s < P.n_splits; ++s) M = fmaxf(M, P.part_m[((size_t)s * P.B + b) * P.H + h]);
+    float Lsum = 0.f;
     for (int s = 0; s < P.n_splits; ++s) {
       const size_t i = ((size_t)s * P.B + b) * P.H + h;
-      const float ms = P.part_m[i];
-      if (ms != -INFINITY) a += P.part_acc[i * dc + c] * fast_exp2(ms - M);
+      if (P.part_m[i] != -INFINITY) Lsum += P.part_l[i] * fast_exp2(P.part_m[i] - M);
     }
-    chat[c] = a * inv;
+    const float inv = 1.f / Lsum;
+    for (int c = threadIdx.x; c < dc; c += 128) {
+      float a = 0.f;
+      for (int s = 0; s < P.n_splits; ++s) {
+        const size_t i = ((size_t)s * P.B + b) * P.H + h;
+        const float ms = P.part_m[i];
+        if (ms != -INFINITY) a += P.part_acc[i * dc + c] * fast_exp2(ms - M);
+      }
+      chat[bb * dc + c] = a * inv;
+    }
+    if (threadIdx.x == 0 && P.lse2) P.lse2[(size_t)b * P.H + h] = M + __log2f(Lsum);
   }
-  if (threadIdx.x == 0 && P.lse2) P.lse2[(size_t)b * P.H + h] = M + __log2f(Lsum);
   __syncthreads();
   const int i = threadIdx.x;
   const uint16_t *w = P.Wv + ((size_t)h * HD + i) * dc;
-  float o = 0.f;
+  float o[CB];
+#pragma unroll
+  for (int bb = 0; bb < CB; ++bb) o[bb] = 0.f;
   for (int c = 0; c < dc; c += 8) {
     const uint4 v = *reinterpret_cast<const uint4 *>(w + c);
     const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      o = fmaf(__uint_as_float(ww[e] << 16), chat[c + 2 * e], o);
-      o = fmaf(__uint_as_float(ww[e] & 0xFFFF0000u), chat[c + 2 * e + 1], o);
+      const float w0 = __uint_as_float(ww[e] << 16), w1 = __uint_as_float(ww[e] & 0xFFFF0000u);
+#pragma unroll
+      for (int bb = 0; bb < CB; ++bb) {
+        if (bb < nb) {
+          o[bb] = fmaf(w0, chat[bb * dc + c + 2 * e], o[bb]);
+          o[bb] = fmaf(w1, chat[bb * dc + c + 2 * e + 1], o[bb]);
+        }
+      }
     }
   }
-  const size_t oi = (size_t)b * P.H * HD + (size_t)h * HD + i;
-  if (P.G) o *= sigmoidf_(bf16_to_f32(P.G[oi]));
-  P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+#pragma unroll
+  for (int bb = 0; bb < CB; ++bb) {
+    if (bb < nb) {
+      const size_t oi = (size_t)(b0 + bb) * P.H * HD + (size_t)h * HD + i;
+      float r = o[bb];
+      if (P.G) r *= sigmoidf_(bf16_to_f32(P.G[oi]));
+      P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+    }
+  }
 }
 
 __global__ void weights_fix_kernel(float *w, const float *lse2, int BH, int L) {
@@ -205,32 +134,52 @@ __global__ void weights_fix_kernel(float *w, const float *lse2, int BH, int L) {
 
 }  // namespace latent
 
-// Workspace layout (bytes, each region 256-aligned):
-//   q~  float [B,H,dc] | m, l float [S,B,H] each | acc float [S,B,H,dc] | lse2 float [B,H]
+// ------------------------------------------------------------------ split planning and workspace
+
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int latent_num_splits(long long B, long long L) {
-  // enough CTAs (splits x head groups x batches) to fill the GPU a few times
-  long long s = (4LL * num_sms() + B * 12 - 1) / (B * 12);
-  if (s < 1) s = 1;
-  long long max_s = (L + 255) / 256;
-  if (s > max_s) s = max_s;
-  if (s > 256) s = 256;
-  return (int)s;
+// Split count for B sequences of L keys: fill whole waves of the 148 SMs of a
+// B200 (one CTA per SM) while keeping the float32 partial states small next to
+// the cache.  A pure function of (B, L) so the workspace size never depends on
+// the device.
+void latent_plan(long long B, long long L, int *n_splits, int *keys_per_split) {
+  const int KT = latent_tc_tile_keys();
+  const long long tiles = (L + KT - 1) / KT;
+  double best = 1e30;
+  long long best_s = 1;
+  for (long long s = 1; s <= 64 && s <= tiles; ++s) {
+    const long long ctas = B * s;
+    const long long waves = (ctas + 147) / 148;
+    const double eff = (double)ctas / (double)(waves * 148);
+    const double overhead = (double)s * 96 * 512 * 8 / ((double)L * 512 * 2 + 1.0);
+    const double cost = 1.0 / eff + overhead;
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_s = s;
+    }
+  }
+  long long kps = ((tiles + best_s - 1) / best_s) * KT;
+  long long s = (L + kps - 1) / kps;  // no empty split
+  *n_splits = (int)s;
+  *keys_per_split = (int)kps;
 }
 
+// Workspace layout (each region 256-byte aligned):
+//   q~ bf16 [B,H,dc] | m, l float [S,B,H] each | acc float [S,B,H,dc] | lse2 float [B,H]
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc) {
-  const long long S = latent_num_splits(B, L);
-  return align256(sizeof(float) * B * H * dc) + 2 * align256(sizeof(float) * S * B * H) +
-         align256(sizeof(float) * S * B * H * dc) + align256(sizeof(float) * B * H);
+  int S, kps;
+  latent_plan(B, L, &S, &kps);
+  return align256(2 * B * H * dc) + 2 * align256(sizeof(float) * S * B * H) + align256(sizeof(float) * S * B * H * dc) +
+         align256(sizeof(float) * B * H);
 }
 
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
   using namespace latent;
-  const int S = latent_num_splits(a.B, a.L);
+  int S, kps;
+  latent_plan(a.B, a.L, &S, &kps);
   uint8_t *ws = static_cast<uint8_t *>(a.workspace);
-  float *qt = reinterpret_cast<float *>(ws);
-  ws += align256(sizeof(float) * a.B * a.H * a.dc);
+  uint16_t *qt = reinterpret_cast<uint16_t *>(ws);
+  ws += align256(2 * (size_t)a.B * a.H * a.dc);
   float *pm = reinterpret_cast<float *>(ws);
   ws += align256(sizeof(float) * (size_t)S * a.B * a.H);
   float *pl = reinterpret_cast<float *>(ws);
@@ -239,30 +188,24 @@ int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
   ws += align256(sizeof(float) * (size_t)S * a.B * a.H * a.dc);
   float *lse2 = reinterpret_cast<float *>(ws);
 
-  const float sl2 = a.scale * kLog2e;
   {
     const size_t shm = sizeof(float) * a.B * HD;
-    if (shm > 48 * 1024) cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
-    absorb_kernel<<<dim3(a.H, (a.dc + 127) / 128), 128, shm, stream>>>(a.Q, a.Wk, a.B, a.H, a.dc, sl2, qt);
+    if (shm > 48 * 1024 &&
+        cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm) != cudaSuccess)
+      return -1;
+    absorb_kernel<<<dim3(a.H, (a.dc + 127) / 128), 128, shm, stream>>>(a.Q, a.Wk, a.B, a.H, a.dc,
+                                                                      a.scale * kLog2e, qt);
   }
   {
-    StreamParams P;
-    P.C = a.C;
-    P.cache_len_max = a.cache_len_max;
-    P.L = a.L;
-    P.H = a.H;
-    P.dc = a.dc;
-    P.n_splits = S;
-    P.keys_per_split = (int)(((a.L + S - 1) / S + KT - 1) / KT * KT);
-    P.qt = qt;
-    P.part_m = pm;
-    P.part_l = pl;
-    P.part_acc = pacc;
-    P.weights = a.weights;
-    P.B = a.B;
-    const size_t shm = sizeof(float) * ((size_t)HG * a.dc + (size_t)KT * a.dc + HG * KT + 2 * HG);
-    cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
-    stream_kernel<<<dim3(S, (a.H + HG - 1) / HG, a.B), ST, shm, stream>>>(P);
+    CUtensorMap tq, tc;
+    const long long dq[3] = {a.dc, a.H, a.B}, sq[2] = {a.dc, (long long)a.H * a.dc};
+    const unsigned bq[3] = {64, 96, 1};
+    if (!make_tmap_bf16(&tq, qt, 3, dq, sq, bq)) return -1;
+    const long long dcm[3] = {a.dc, a.cache_len_max, a.B}, scm[2] = {a.dc, a.cache_len_max * a.dc};
+    const unsigned bc[3] = {64, (unsigned)latent_tc_tile_keys(), 1};
+    if (!make_tmap_bf16(&tc, a.C, 3, dcm, scm, bc)) return -1;
+    if (launch_latent_tc(tq, tc, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, a.status, stream) != 0)
+      return -1;
   }
   {
     CombineParams P;
@@ -277,7 +220,7 @@ int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
     P.G = a.G;
     P.O = a.O;
     P.lse2 = lse2;
-    combine_kernel<<<dim3(a.H, a.B), 128, sizeof(float) * a.dc, stream>>>(P);
+    combine_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), 128, sizeof(float) * CB * a.dc, stream>>>(P);
   }
   if (a.weights) weights_fix_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, a.B * a.H, a.L);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

@@ -71,7 +71,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 // bf16 tiled map with 128-byte swizzle.  dims/strides in elements, dim 0 innermost (contiguous).
-static bool make_map(CUtensorMap *m, const void *base, int rank, const long long *dims, const long long *strides,
+bool make_tmap_bf16(CUtensorMap *m, const void *base, int rank, const long long *dims, const long long *strides,
                      const unsigned *box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -158,7 +158,7 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
     CUtensorMap tmA, tmB[3];
     const long long dA[3] = {d_model, M, 1}, sA[2] = {d_model, M * d_model};
     const unsigned bA[3] = {64, 128, 1};
-    if (!make_map(&tmA, X, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+    if (!make_tmap_bf16(&tmA, X, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
     ga.a_rows = (int)M;
     ga.a_batches = 1;
     ga.a_row0 = 0;
@@ -172,7 +172,7 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
       const long long N = i == 2 ? d_c : d_model;
       const long long dB[2] = {d_model, N}, sB[1] = {d_model};
       const unsigned bB[2] = {64, 256};
-      if (!make_map(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+      if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
       GemmOut &o = ga.prob[np];
       o.out = Os[i];
       o.N = (int)N;
@@ -198,7 +198,7 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
     CUtensorMap tmA, tmB[3];
     const long long dA[3] = {d_c, cache_pos + T, B}, sA[2] = {d_c, cache_len_max * d_c};
     const unsigned bA[3] = {64, 128, 1};
-    if (!make_map(&tmA, C, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+    if (!make_tmap_bf16(&tmA, C, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
     ga.a_rows = (int)T;
     ga.a_batches = (int)B;
     ga.a_row0 = (int)cache_pos;
@@ -211,7 +211,7 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
       if (!Os[i]) continue;
       const long long dB[2] = {d_c, d_model}, sB[1] = {d_c};
       const unsigned bB[2] = {64, 256};
-      if (!make_map(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+      if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
       GemmOut &o = ga.prob[np];
       o.out = Os[i];
       o.N = (int)d_model;
@@ -266,15 +266,15 @@ gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_strides[3], 
   const unsigned box[4] = {64, 128, 1, 1};
   {
     const long long d[4] = {128, Tq, H, B}, sd[3] = {q_strides[1], q_strides[2], q_strides[0]};
-    if (!make_map(&tq, Q, 4, d, sd, box)) return GMLA_ERR_CUDA;
+    if (!make_tmap_bf16(&tq, Q, 4, d, sd, box)) return GMLA_ERR_CUDA;
   }
   {
     const long long d[4] = {128, Tk, H, B}, sd[3] = {k_strides[1], k_strides[2], k_strides[0]};
-    if (!make_map(&tk, K, 4, d, sd, box)) return GMLA_ERR_CUDA;
+    if (!make_tmap_bf16(&tk, K, 4, d, sd, box)) return GMLA_ERR_CUDA;
   }
   {
     const long long d[4] = {128, Tk, H, B}, sd[3] = {v_strides[1], v_strides[2], v_strides[0]};
-    if (!make_map(&tv, V, 4, d, sd, box)) return GMLA_ERR_CUDA;
+    if (!make_tmap_bf16(&tv, V, 4, d, sd, box)) return GMLA_ERR_CUDA;
   }
   PrefillArgs a{};
   a.G = G; a.O = O;
@@ -301,7 +301,7 @@ gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B
   const void *ptrs[] = {Q, C, W_k, W_v, G, O, workspace};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return GMLA_ERR_ARG;
-  if (D_h != 128 || d_c % 64 != 0 || d_c > 512) return GMLA_ERR_UNSUPPORTED;
+  if (D_h != 128 || d_c % 64 != 0 || d_c > 512 || H > 96) return GMLA_ERR_UNSUPPORTED;
   if (B > 65535 || H > 65535 || L > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
   const size_t need = latent_workspace_bytes(B, L, H, d_c);
   if (!workspace || workspace_bytes < need) return GMLA_ERR_WORKSPACE;
@@ -336,10 +336,10 @@ gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf1
   CUtensorMap tmA, tmB[3];
   const long long dA[3] = {d_model, M, 1}, sA[2] = {d_model, M * d_model};
   const unsigned bA[3] = {64, 128, 1};
-  if (!make_map(&tmA, O, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+  if (!make_tmap_bf16(&tmA, O, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
   const long long dB[2] = {d_model, d_model}, sB[1] = {d_model};
   const unsigned bB[2] = {64, 256};
-  if (!make_map(&tmB[0], W_o, 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+  if (!make_tmap_bf16(&tmB[0], W_o, 2, dB, sB, bB)) return GMLA_ERR_CUDA;
   ga.a_rows = (int)M;
   ga.a_batches = 1;
   ga.a_row0 = 0;

@@ -77,4 +77,8 @@ size_t latent_workspace_bytes(long long B, long long L, long long H, long long d
 
 int num_sms();
 
+// bf16 TMA tensor map with 128-byte swizzle; dims/strides in elements, dim 0 contiguous.
+bool make_tmap_bf16(CUtensorMap *m, const void *base, int rank, const long long *dims, const long long *strides,
+                    const unsigned *box);
+
 }  // namespace gmla

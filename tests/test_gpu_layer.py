@@ -109,6 +109,30 @@ def test_attend_decode_matches_oracle(g, B, L, Lmax, H, d_c):
     assert np.abs(w - wref).max() < 1e-4
 
 
+def test_attend_decode_full_size_sampled(g):
+    """Latent-cache decode at the timed size: B=32, L=131072, d_c=512, 96 heads;
+    checked on sampled (b, h) pairs (the oracle rebuilds K_h, V_h from the cache)."""
+    B, L, H, d_c = 32, 131072, 96, 512
+    d = 128 * H
+    dr = Draw(SEEDS["latent_decode"] + 100)
+    q = dr.normal((B, d))
+    Wk = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Wv = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Gl = dr.normal((B, d))
+    cache = dr.normal((B, L, d_c))
+    Cd = to_dev(cache)
+    O = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    work = ws(g.gmla_attend_decode_workspace_size(B, L, H, d_c))
+    g.gmla_attend_decode(to_dev(q), Cd, L, to_dev(Wk), to_dev(Wv), O, H, G=to_dev(Gl), workspace=work)
+    g.gmla_get_device_status()
+    pairs = [(0, 0), (31, 95), (7, 48), (19, 3)]
+    ref = orc.decode_latent(q, cache, L, Wk, Wv, H, G=Gl, heads=pairs)
+    got = f64(O)
+    sel = np.concatenate([np.arange(h * 128, (h + 1) * 128) + b * d for b, h in pairs])
+    assert_parity(got.reshape(-1)[sel], ref.reshape(-1)[sel], "decode full-size sampled heads")
+    assert np.all(np.isfinite(got))
+
+
 def test_decode_equals_prefill_last_row(g):
     """Decode of token t over latents 0..t equals row t of causal prefill (same GPU inputs)."""
     B, T, H, d_c = 1, 257, 2, 128
