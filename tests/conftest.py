@@ -13,6 +13,16 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+    # both native libraries are built in-tree (no-ops when up to date); the build
+    # script is loaded by path because the package itself needs the built library
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_gmla_build", os.path.join(ROOT, "causal_head_latent_b200",
+                                                                              "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    from oracle import build as ob
+    ob.build()
 
 
 def pytest_collection_modifyitems(config, items):
