@@ -48,14 +48,17 @@ def prefill_flops(B=P_B, H=P_H, T=P_T):
     return 4.0 * D * H * B * T * (T + 1) / 2
 
 
-def decode_bytes(B=DEC_B, L=DEC_L, H=96, dc=DC):
+def decode_bytes(B=None, L=None, H=96, dc=DC):
     # algorithmic bytes of gmla_attend_decode: the visible latents, W_k, W_v, q, G and O
+    B = DEC_B if B is None else B
+    L = DEC_L if L is None else L
     d = H * D
     return 2.0 * (B * L * dc + 2 * d * dc + 3 * B * d)
 
 
-def decode_step_bytes(B=DEC_B, L=DEC_L, dc=DC, dm=DM):
+def decode_step_bytes(B=None, L=None, dc=DC, dm=DM):
     # whole decode step: attend_decode plus W_q, W_g, W_c, W_o and the new-token activations
+    B = DEC_B if B is None else B
     return decode_bytes(B, L, dm // D, dc) + 2.0 * (3 * dm * dm + dc * dm + 4 * B * dm + B * dc)
 
 
@@ -400,7 +403,11 @@ def main():
     ap.add_argument("--workload", default="step", choices=["step", "layer"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--dec-L", type=int, default=DEC_L,
+                    help="cached latent length of the decode part (smaller only for profiling captures)")
     args = ap.parse_args()
+    global DEC_L
+    DEC_L = args.dec_L
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
 

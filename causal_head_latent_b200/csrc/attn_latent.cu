@@ -16,9 +16,9 @@
 
 namespace gmla {
 
-int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, int B, int L, int H, int dc, int n_splits,
-                     int keys_per_split, float *part_m, float *part_l, float *part_acc, float *weights,
-                     unsigned *status, cudaStream_t stream);
+int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
+                     int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l, float *part_acc,
+                     float *weights, unsigned *status, cudaStream_t stream);
 int latent_tc_tile_keys();
 
 namespace latent {
@@ -204,7 +204,7 @@ int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
     const long long dcm[3] = {a.dc, a.cache_len_max, a.B}, scm[2] = {a.dc, a.cache_len_max * a.dc};
     const unsigned bc[3] = {64, (unsigned)latent_tc_tile_keys(), 1};
     if (!make_tmap_bf16(&tc, a.C, 3, dcm, scm, bc)) return -1;
-    if (launch_latent_tc(tq, tc, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, a.status, stream) != 0)
+    if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, a.status, stream) != 0)
       return -1;
   }
   {

@@ -34,6 +34,7 @@ constexpr int QCHUNK = HMAX * 128;         // 12 KB
 constexpr int Q_BYTES = 8 * QCHUNK + 4096; // + tail read by the padded rows of the last chunk
 constexpr int P_BYTES = HMAX * 128;        // P^T rows: one 128-byte swizzled row per head
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kPrefetchTiles = 8;          // L2 prefetch distance of the latent stream
 constexpr int TM_S = 0;                    // two S buffers of 64 columns
 constexpr int TM_ACC = 128;                // acc^T blocks: 128 + 96*blk
 
@@ -44,6 +45,8 @@ struct Geo {
 };
 
 struct Params {
+  const uint16_t *C;  // latent cache [B, Lmax, dc] (for the L2 prefetch stream)
+  long long Lmax;
   int B, L, H, dc, n_splits, keys_per_split;
   float *part_m, *part_l, *part_acc;  // [S,B,H], [S,B,H], [S,B,H,512]
   float *weights;                     // optional raw log2-domain scores [B,H,L]
@@ -135,8 +138,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tmC);
       mbar_arrive_expect_tx(bar_q, 8 * QCHUNK);
       for (int kc = 0; kc < 8; ++kc) tma_load_3d(sq + kc * QCHUNK, &tmQt, bar_q, kc * 64, 0, b);
+      // The latents of this split are one contiguous range; keep an L2 prefetch
+      // stream kPrefetchTiles ahead of the shared-memory ring so DRAM latency is
+      // hidden without more shared memory.
+      const uint8_t *crow = reinterpret_cast<const uint8_t *>(p.C + ((size_t)b * p.Lmax) * p.dc);
+      const size_t key_bytes = (size_t)p.dc * 2;
+      auto prefetch_tile = [&](int jt) {
+        const int kb = k_begin + jt * KT;
+        if (jt < n_tiles) prefetch_l2_bulk(crow + (size_t)kb * key_bytes, (uint32_t)(min(KT, k_end - kb) * key_bytes));
+      };
+      for (int jt = 1; jt < kPrefetchTiles; ++jt) prefetch_tile(jt);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % STAGES;
+        prefetch_tile(j + kPrefetchTiles);
         if (!mbar_wait(&c_empty[s], ((j / STAGES) & 1) ^ 1, p.status)) break;
         mbar_arrive_expect_tx(&c_full[s], G::C_BYTES);
         uint8_t *dst = sc + s * G::C_BYTES;
@@ -320,14 +334,14 @@ size_t smem_bytes() {
 }  // namespace latent_tc
 
 // Keys per tile and pipeline depth of the tensor-core decode.
-constexpr int kLatentKT = 48;
-constexpr int kLatentStages = 2;
+constexpr int kLatentKT = 32;
+constexpr int kLatentStages = 3;
 
 int latent_tc_tile_keys() { return kLatentKT; }
 
-int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, int B, int L, int H, int dc, int n_splits,
-                     int keys_per_split, float *part_m, float *part_l, float *part_acc, float *weights,
-                     unsigned *status, cudaStream_t stream) {
+int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
+                     int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l, float *part_acc,
+                     float *weights, unsigned *status, cudaStream_t stream) {
   using namespace latent_tc;
   auto kern = latent_decode_kernel<kLatentKT, kLatentStages>;
   const size_t smem = smem_bytes<kLatentKT, kLatentStages>();
@@ -337,6 +351,8 @@ int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, int B, int
     configured = true;
   }
   Params p;
+  p.C = C;
+  p.Lmax = Lmax;
   p.B = B;
   p.L = L;
   p.H = H;

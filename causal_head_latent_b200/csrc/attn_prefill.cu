@@ -5,19 +5,23 @@
 // page, "Start from familiar attention"; "Kimi K3 - Softmax over keys";
 // mask of "Kimi K2 - Construct causal mask").  Query t of Tq sits at absolute
 // position Tk - Tq + t.  The softmax runs online over key tiles (running max
-// and sum with rescaling, Milakov & Gimelshein 2018), which is exact in real
-// arithmetic.
+// and sum with rescaling, Milakov & Gimelshein 2018), exact in real arithmetic.
 //
-// One CTA owns one 128-row query tile of one (b, h):
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
-//   warp 1      TMEM owner and MMA issuer (one thread):
-//                 S = Q K^T   (M=128, N=128, K=128, both operands K-major)
-//                 O += P V    (P from shared memory, V MN-major)
-//   warps 2..5  softmax warpgroup, one query row per thread (TMEM lane):
-//                 S row from TMEM, mask, online max/sum in the exp2 domain,
-//                 P row (bf16) into shared memory, O rescale in TMEM when the
-//                 running max grows by more than 2^8, final 1/l, gate, store.
-// TMEM: S in columns [0,128), O in [128,256).
+// One CTA owns two 128-row query tiles (Q0, Q1) of one (b, h) and streams the
+// K/V tiles they need once for both:
+//   warp 0      TMA producer: Q0, Q1, then K and V tiles into 2-stage rings
+//   warp 1      TMEM owner and MMA issuer (one thread).  Per key tile j the
+//               tensor core runs   PV0_j, S0_{j+1}, PV1_j, S1_{j+1}
+//               with S_i = Q_i K^T (both operands K-major, in shared memory)
+//               and O_i += P_i V (P_i read from TMEM, V MN-major in shared
+//               memory), so softmax of one tile overlaps MMAs of the other.
+//   warps 2-5   softmax warpgroup of Q0, one query row per thread (TMEM lane)
+//   warps 6-9   softmax warpgroup of Q1
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  P_i
+// (bfloat16, two per column) overwrites the first 64 columns of S_i.
+// Because S_i of tile j+1 is issued after PV_i of tile j, its completion also
+// means PV_i_j is done: the softmax may then rescale O_i (lazy: only when the
+// running max grew by more than 2^8) and overwrite P_i without further waits.
 // Tiles above the diagonal are skipped; only diagonal / tail tiles are masked.
 #include "internal.h"
 #include "ptx.cuh"
@@ -25,33 +29,28 @@
 namespace gmla {
 namespace prefill {
 
-constexpr int BM = 128;           // query rows per CTA
-constexpr int BN = 128;           // keys per tile
-constexpr int HD = 128;           // head dimension
-constexpr int STAGES = 2;         // K/V ring depth
-constexpr int TILE_BYTES = BM * HD * 2;  // one 128x128 bf16 operand tile = 2 swizzled 64-column chunks
+constexpr int BM = 128;                  // query rows per tile
+constexpr int BN = 128;                  // keys per tile
+constexpr int HD = 128;                  // head dimension
+constexpr int STAGES = 2;                // K and V ring depth
+constexpr int TILE_BYTES = BM * HD * 2;  // 128 x 128 bf16 = two 64-column swizzled chunks
 constexpr int CHUNK_BYTES = TILE_BYTES / 2;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p we let through unrescaled
+constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p let through unrescaled
 
 struct Smem {
-  uint8_t q[TILE_BYTES];
+  uint8_t q[2][TILE_BYTES];
   uint8_t k[STAGES][TILE_BYTES];
   uint8_t v[STAGES][TILE_BYTES];
-  uint8_t p[TILE_BYTES];
   uint64_t bar_q;
-  uint64_t bar_k_full[STAGES];
-  uint64_t bar_v_full[STAGES];
-  uint64_t bar_kv_empty[STAGES];
-  uint64_t bar_s_full;
-  uint64_t bar_s_free;
-  uint64_t bar_p_full;
-  uint64_t bar_o_done;
+  uint64_t k_full[STAGES], k_empty[STAGES];
+  uint64_t v_full[STAGES], v_empty[STAGES];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
   uint32_t tmem_base;
-  int abort_flag;
 };
-
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
 
 struct Params {
@@ -61,59 +60,82 @@ struct Params {
   float *lse;
   float *weights;
   int B, H, Tq, Tk, causal;
-  int n_qt;
+  int n_ct;          // CTAs (256-row query pairs) per (b, h)
   float scale_log2;  // scale * log2(e)
   unsigned *status;
 };
 
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t addr) { return sdesc_sw128(addr, 16, 1024); }
 
+// D[tmem] (+)= A[tmem] * B[smem] (A from tensor memory, K-major).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Number of key tiles query tile `qt` needs (0 when the tile has no valid row).
+__device__ __forceinline__ int kv_tiles(const Params &p, int qt) {
+  const int q0 = qt * BM;
+  if (q0 >= p.Tq) return 0;
+  const int last_row = min(q0 + BM - 1, p.Tq - 1);
+  const int last_key = p.causal ? min(p.Tk - 1, p.Tk - p.Tq + last_row) : (p.Tk - 1);
+  return last_key / BN + 1;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // Heavy (late) query tiles first; consecutive CTAs take different heads.
-  const int BH = p.B * p.H;
-  const int lin = blockIdx.x;
-  const int qt = p.causal ? (p.n_qt - 1 - lin / BH) : (lin / BH);
-  const int bh = lin % BH;
+  // Head-major CTA order (the K/V of the few heads in flight stay in L2); within
+  // a head the longest (latest) query pairs first.
+  const int bh = blockIdx.x / p.n_ct;
+  const int ct = p.causal ? (p.n_ct - 1 - blockIdx.x % p.n_ct) : (blockIdx.x % p.n_ct);
   const int b = bh / p.H, h = bh % p.H;
-  const int q0 = qt * BM;
-  const int shift = p.Tk - p.Tq;  // absolute position of query 0
-  // Keys needed by this tile: 0 .. last_key
-  const int last_row = min(q0 + BM - 1, p.Tq - 1);
-  const int last_key = p.causal ? min(p.Tk - 1, shift + last_row) : (p.Tk - 1);
-  const int n_kv = last_key / BN + 1;
+  const int nkv0 = kv_tiles(p, 2 * ct);
+  const int nkv1 = kv_tiles(p, 2 * ct + 1);
+  const int nkv = max(nkv0, nkv1);
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.bar_k_full[s], 1);
-      mbar_init(&sm.bar_v_full[s], 1);
-      mbar_init(&sm.bar_kv_empty[s], 1);
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
-    mbar_init(&sm.bar_s_full, 1);
-    mbar_init(&sm.bar_s_free, 4);
-    mbar_init(&sm.bar_p_full, 4);
-    mbar_init(&sm.bar_o_done, 1);
-    sm.abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 4);
+    }
+    mbar_init(&sm.o_done, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 256);
+    tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tS = tmem;
-  const uint32_t tO = tmem + 128;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -121,19 +143,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&sm.bar_q, TILE_BYTES);
-      tma_load_4d(sm.q, &tmQ, &sm.bar_q, 0, q0, h, b);
-      tma_load_4d(sm.q + CHUNK_BYTES, &tmQ, &sm.bar_q, 64, q0, h, b);
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % STAGES, r = j / STAGES;
-        if (!mbar_wait(&sm.bar_kv_empty[s], (r & 1) ^ 1, p.status)) { sm.abort_flag = 1; break; }
+      const int q0 = 2 * ct * BM;
+      mbar_arrive_expect_tx(&sm.bar_q, 2 * TILE_BYTES);
+      for (int i = 0; i < 2; ++i) {
+        tma_load_4d(sm.q[i], &tmQ, &sm.bar_q, 0, q0 + i * BM, h, b);
+        tma_load_4d(sm.q[i] + CHUNK_BYTES, &tmQ, &sm.bar_q, 64, q0 + i * BM, h, b);
+      }
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % STAGES, ph = ((j / STAGES) & 1) ^ 1;
         const int k0 = j * BN;
-        mbar_arrive_expect_tx(&sm.bar_k_full[s], TILE_BYTES);
-        tma_load_4d(sm.k[s], &tmK, &sm.bar_k_full[s], 0, k0, h, b);
-        tma_load_4d(sm.k[s] + CHUNK_BYTES, &tmK, &sm.bar_k_full[s], 64, k0, h, b);
-        mbar_arrive_expect_tx(&sm.bar_v_full[s], TILE_BYTES);
-        tma_load_4d(sm.v[s], &tmV, &sm.bar_v_full[s], 0, k0, h, b);
-        tma_load_4d(sm.v[s] + CHUNK_BYTES, &tmV, &sm.bar_v_full[s], 64, k0, h, b);
+        if (!mbar_wait(&sm.k_empty[s], ph, p.status)) break;
+        mbar_arrive_expect_tx(&sm.k_full[s], TILE_BYTES);
+        tma_load_4d(sm.k[s], &tmK, &sm.k_full[s], 0, k0, h, b);
+        tma_load_4d(sm.k[s] + CHUNK_BYTES, &tmK, &sm.k_full[s], 64, k0, h, b);
+        if (!mbar_wait(&sm.v_empty[s], ph, p.status)) break;
+        mbar_arrive_expect_tx(&sm.v_full[s], TILE_BYTES);
+        tma_load_4d(sm.v[s], &tmV, &sm.v_full[s], 0, k0, h, b);
+        tma_load_4d(sm.v[s] + CHUNK_BYTES, &tmV, &sm.v_full[s], 64, k0, h, b);
       }
     }
   } else if (warp == 1) {
@@ -141,98 +167,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 128, false, true);
-      const uint32_t aQ = smem_u32(sm.q);
-      const uint32_t aP = smem_u32(sm.p);
+      const uint32_t aQ[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      const int nk[2] = {nkv0, nkv1};
       bool ok = mbar_wait(&sm.bar_q, 0, p.status);
-      for (int j = 0; ok && j <= n_kv; ++j) {
-        if (j < n_kv) {
-          const int s = j % STAGES;
-          ok = mbar_wait(&sm.bar_k_full[s], (j / STAGES) & 1, p.status);
-          if (ok && j > 0) ok = mbar_wait(&sm.bar_s_free, (j - 1) & 1, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t aK = smem_u32(sm.k[s]);
+      // S_i for key tile j (K-major Q_i and K_j)
+      auto issue_s = [&](int i, int j) {
+        const uint32_t aK = smem_u32(sm.k[j % STAGES]);
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-            umma_bf16_ss(tS, desc_kmajor(aQ + off), desc_kmajor(aK + off), idS, kk > 0);
-          }
-          umma_commit(&sm.bar_s_full);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
+          umma_bf16_ss(tmem + i * 128, desc_kmajor(aQ[i] + off), desc_kmajor(aK + off), idS, kk > 0);
         }
-        if (j > 0) {
-          const int jp = j - 1, s = jp % STAGES;
-          ok = mbar_wait(&sm.bar_p_full, jp & 1, p.status);
-          if (ok) ok = mbar_wait(&sm.bar_v_full[s], (jp / STAGES) & 1, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t aV = smem_u32(sm.v[s]);
+        umma_commit(&sm.s_full[i]);
+      };
+      // O_i += P_i V_j (P_i in TMEM columns [128 i, 128 i + 64), V_j MN-major)
+      auto issue_pv = [&](int i, int j) {
+        const uint32_t aV = smem_u32(sm.v[j % STAGES]);
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t offP = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-            // V tile: rows = keys (128 B per row), two 64-wide D chunks 16 KB apart.
-            umma_bf16_ss(tO, desc_kmajor(aP + offP), sdesc_sw128(aV + kk * 2048, CHUNK_BYTES, 1024), idPV,
-                         (jp > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&sm.bar_o_done);
-          umma_commit(&sm.bar_kv_empty[s]);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
+                       sdesc_sw128(aV + kk * 2048, CHUNK_BYTES, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      if (ok) ok = mbar_wait(&sm.k_full[0], 0, p.status);
+      if (ok) {
+        tc_fence_after();
+        for (int i = 0; i < 2; ++i)
+          if (nk[i] > 0) issue_s(i, 0);
+        umma_commit(&sm.k_empty[0]);
       }
-      if (!ok) sm.abort_flag = 1;
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % STAGES;
+        const bool next = j + 1 < nkv;
+        ok = mbar_wait(&sm.v_full[s], (j / STAGES) & 1, p.status);
+        if (ok && next) ok = mbar_wait(&sm.k_full[(j + 1) % STAGES], ((j + 1) / STAGES) & 1, p.status);
+        for (int i = 0; ok && i < 2; ++i) {
+          if (j < nk[i]) {
+            if (!(ok = mbar_wait(&sm.p_full[i], j & 1, p.status))) break;
+            tc_fence_after();
+            issue_pv(i, j);
+          }
+          if (j + 1 < nk[i]) issue_s(i, j + 1);
+        }
+        if (!ok) break;
+        umma_commit(&sm.v_empty[s]);
+        if (next) umma_commit(&sm.k_empty[(j + 1) % STAGES]);
+      }
+      if (ok) umma_commit(&sm.o_done);
     }
   } else {
-    // ---------------------------------------------------------------- softmax warpgroup
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int wg = (warp - 2) >> 2;         // 0: Q0, 1: Q1
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // query row within the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int t = q0 + row;                 // query index
+    const uint32_t tS = tmem + wg * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + wg * 128 + lane_off;
+    const int n_tiles = wg ? nkv1 : nkv0;
+    const int q0 = (2 * ct + wg) * BM;
+    const int t = q0 + row;
     const bool row_valid = t < p.Tq;
-    const int pos = shift + t;              // absolute position
+    const int shift = p.Tk - p.Tq;
+    const int pos = shift + t;
+    const int lim = p.causal ? min(pos, p.Tk - 1) : (p.Tk - 1);  // last visible key of this row
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     float *wrow = (p.weights && row_valid) ? p.weights + (((size_t)b * p.H + h) * p.Tq + t) * (size_t)p.Tk : nullptr;
-    uint8_t *prow = sm.p + row * 128;
-    const int sw = row & 7;
     bool ok = true;
 
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < n_tiles; ++j) {
       const int k0 = j * BN;
-      if (!mbar_wait(&sm.bar_s_full, j & 1, p.status)) { ok = false; break; }
+      if (!mbar_wait(&sm.s_full[wg], j & 1, p.status)) { ok = false; break; }
       tc_fence_after();
       float x[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         float tmp[32];
-        tmem_ld32(tS + lane_off + c * 32, tmp);
+        tmem_ld32(tS + c * 32, tmp);
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[c * 32 + i] = tmp[i];
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.bar_s_free);
-
-      // scale into the log2 domain, mask, row max
       const bool need_mask = (k0 + BN > p.Tk) || (p.causal && (k0 + BN - 1 > shift + q0));
-      float mx = -INFINITY;
       if (need_mask) {
-        const int lim = p.causal ? min(pos, p.Tk - 1) : (p.Tk - 1);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          x[c] = (k0 + c <= lim) ? x[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, x[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          x[c] *= sl2;
-          mx = fmaxf(mx, x[c]);
-        }
+        for (int c = 0; c < BN; ++c)
+          if (k0 + c > lim) x[c] = -INFINITY;
       }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      mx *= sl2;  // scale > 0 commutes with max
       if (wrow) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
-          if (k0 + c < p.Tk) wrow[k0 + c] = x[c];
+          if (k0 + c < p.Tk) wrow[k0 + c] = x[c] * sl2;
       }
-      // lazy rescale: keep the old reference max unless this tile exceeds it by > 2^8
+      // lazy rescale: keep the reference max unless this tile exceeds it by > 2^8
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_used + kRescaleThreshold) {
@@ -242,48 +271,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         m_used = mx;
       }
-      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      const float nref = (m_used == -INFINITY) ? 0.f : -m_used;
       float rs = 0.f;
-      uint32_t pk[BN / 2];
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = fast_exp2(x[c] - mref);
-        const float p1 = fast_exp2(x[c + 1] - mref);
-        rs += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = fast_exp2(fmaf(x[c + e], sl2, nref));
+          const float p1 = fast_exp2(fmaf(x[c + e + 1], sl2, nref));
+          rs += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c / 2, pk);
       }
       l = l * alpha + rs;
-
-      // PV of the previous tile must be done before O is rescaled or P overwritten.
-      if (j > 0) {
-        if (!mbar_wait(&sm.bar_o_done, (j - 1) & 1, p.status)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+      // S_i of this tile completed after PV_i of the previous tile, so O_i is idle here.
+      if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-          for (int c = 0; c < HD / 32; ++c) {
-            float o[32];
-            tmem_ld32(tO + lane_off + c * 32, o);
+        for (int c = 0; c < HD / 32; ++c) {
+          float o[32];
+          tmem_ld32(tO + c * 32, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO + lane_off + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tO + c * 32, o);
         }
       }
-      // P row -> shared memory in the 128-byte-swizzled K-major layout
-#pragma unroll
-      for (int u = 0; u < BN / 8; ++u) {
-        const int chunk = u >> 3, uu = u & 7;
-        uint4 val = make_uint4(pk[u * 4 + 0], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
-        *reinterpret_cast<uint4 *>(prow + chunk * CHUNK_BYTES + ((uu ^ sw) << 4)) = val;
-      }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.bar_p_full);
+      if (lane == 0) mbar_arrive(&sm.p_full[wg]);
     }
 
     // ---------------------------------------------------------------- epilogue
-    if (ok && mbar_wait(&sm.bar_o_done, (n_kv - 1) & 1, p.status)) {
+    if (n_tiles > 0 && ok && mbar_wait(&sm.o_done, 0, p.status)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       uint16_t *orow = p.O + (long long)b * p.o_sb + (long long)t * p.o_st + (long long)h * p.o_sh;
@@ -291,7 +312,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         float o[32];
-        tmem_ld32(tO + lane_off + c * 32, o);
+        tmem_ld32(tO + c * 32, o);
         if (row_valid) {
           if (grow) {
             const uint4 *g4 = reinterpret_cast<const uint4 *>(grow + c * 32);
@@ -319,12 +340,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (row_valid && p.lse) p.lse[((size_t)b * p.H + h) * p.Tq + t] = (m_used + __log2f(l)) * 0.6931471805599453f;
       if (wrow) {
         // debug weights: raw log2-domain scores were stored above; normalise in place
-        const int lim = p.causal ? min(pos, p.Tk - 1) : (p.Tk - 1);
         const float lg = m_used + __log2f(l);
         for (int s = 0; s < p.Tk; ++s) wrow[s] = (s <= lim) ? fast_exp2(wrow[s] - lg) : 0.f;
       }
-    } else {
-      sm.abort_flag = 1;
     }
     tc_fence_before();
   }
@@ -333,7 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -362,10 +380,10 @@ int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CU
   p.Tq = a.Tq;
   p.Tk = a.Tk;
   p.causal = a.causal;
-  p.n_qt = (a.Tq + BM - 1) / BM;
+  p.n_ct = (a.Tq + 2 * BM - 1) / (2 * BM);
   p.scale_log2 = a.scale * kLog2e;
   p.status = a.status;
-  const long long grid = (long long)p.n_qt * a.B * a.H;
+  const long long grid = (long long)p.n_ct * a.B * a.H;
   if (grid <= 0) return 0;
   if (grid > 0x7fffffffLL) return -2;
   attn_prefill_kernel<<<(unsigned)grid, NUM_THREADS, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
