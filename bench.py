@@ -394,6 +394,7 @@ def timed(fn_list, steps, world):
 
 
 def main():
+    global DEC_L
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -406,7 +407,6 @@ def main():
     ap.add_argument("--dec-L", type=int, default=DEC_L,
                     help="cached latent length of the decode part (smaller only for profiling captures)")
     args = ap.parse_args()
-    global DEC_L
     DEC_L = args.dec_L
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
