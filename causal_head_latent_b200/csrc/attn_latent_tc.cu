@@ -90,8 +90,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sq = base;
   uint8_t *sc = sq + Q_BYTES;                 // Q_BYTES is a multiple of 1024
-  uint8_t *sp = sc + STAGES * G::C_BYTES;
-  float *alpha_s = reinterpret_cast<float *>(sp + P_BYTES);
+  uint8_t *sp = sc + STAGES * G::C_BYTES;     // two P^T buffers
+  float *alpha_s = reinterpret_cast<float *>(sp + 2 * P_BYTES);
   uint64_t *bars = reinterpret_cast<uint64_t *>(alpha_s + 128);
   uint64_t *bar_q = bars;
   uint64_t *c_full = bars + 1;
@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *s_full = c_empty + STAGES;  // [2]
   uint64_t *s_free = s_full + 2;        // [2]
   uint64_t *p_full = s_free + 2;
-  uint64_t *o_done = p_full + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
+  uint64_t *pv_done = p_full + 1;       // [2]: PV of tile j arrives on pv_done[j & 1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int b = blockIdx.x / p.n_splits;
@@ -120,7 +120,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&s_free[i], 4);
     }
     mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -193,8 +194,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int ks = 0; ks < KT / 16; ++ks)
               umma_bf16_ss(tmem + TM_ACC + blk * HMAX,
                            sdesc_sw128(cst + 2 * blk * G::CCHUNK + ks * 2048, G::CCHUNK, 1024),
-                           sdesc_sw128(ap + ks * 32, 16, 1024), idPV, (jp > 0 || ks > 0) ? 1u : 0u);
-          umma_commit(o_done);
+                           sdesc_sw128(ap + (jp & 1) * P_BYTES + ks * 32, 16, 1024), idPV,
+                           (jp > 0 || ks > 0) ? 1u : 0u);
+          umma_commit(&pv_done[jp & 1]);
           umma_commit(&c_empty[s]);
         }
       }
@@ -259,10 +261,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       alpha_s[h] = alpha;
       const bool any = bar_or(1, 128, resc);
 
-      if (j > 0) {
-        if (!mbar_wait(o_done, (j - 1) & 1, p.status)) { ok = false; break; }
+      // P^T buffer j&1 was last read by PV_{j-2}; a rescale of acc^T needs PV_{j-1} done.
+      if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j >> 1) & 1) ^ 1, p.status)) { ok = false; break; }
+      if (j > 0 && any) {
+        if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.status)) { ok = false; break; }
         tc_fence_after();
-        if (any) {
+        {
           // acc^T lanes are d_c rows; columns are heads: scale column h by alpha_s[h]
 #pragma unroll 1
           for (int blk = 0; blk < 4; ++blk) {
@@ -280,9 +284,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (any) bar_sync(1, 128);  // alpha_s is rewritten by the next tile
       if (head_ok) {
+        uint8_t *pr = prow + (j & 1) * P_BYTES;
 #pragma unroll
         for (int u = 0; u < KT / 8; ++u)
-          *reinterpret_cast<uint4 *>(prow + ((u ^ sw) << 4)) =
+          *reinterpret_cast<uint4 *>(pr + ((u ^ sw) << 4)) =
               make_uint4(pk[u * 4 + 0], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
       }
       fence_proxy_async_smem();
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 
     // partial state of this split: m, l per head and acc^T
-    if (ok && mbar_wait(o_done, (n_tiles - 1) & 1, p.status)) {
+    if (ok && mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.status)) {
       tc_fence_after();
       const size_t rec = ((size_t)split * p.B + b) * p.H;
       if (head_ok) {
@@ -328,7 +333,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int KT, int STAGES>
 size_t smem_bytes() {
-  return 1024 + Q_BYTES + STAGES * Geo<KT>::C_BYTES + P_BYTES + 128 * 4 + 8 * (1 + 2 * STAGES + 6) + 16;
+  return 1024 + Q_BYTES + STAGES * Geo<KT>::C_BYTES + 2 * P_BYTES + 128 * 4 + 8 * (1 + 2 * STAGES + 7) + 16;
 }
 
 }  // namespace latent_tc
