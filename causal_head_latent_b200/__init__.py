@@ -54,6 +54,11 @@ lib.gmla_attend_decode.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _
 lib.gmla_attend_decode.restype = _st
 lib.gmla_attend_decode_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
 lib.gmla_attend_decode_workspace_size.restype = _sz
+lib.gmla_attend_decode_noalloc.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p,
+                                           _p, _p, _p]
+lib.gmla_attend_decode_noalloc.restype = _st
+lib.gmla_attend_decode_noalloc_max_bytes.argtypes = []
+lib.gmla_attend_decode_noalloc_max_bytes.restype = _sz
 lib.gmla_gate_out.argtypes = [_p, _p, _p, _i64, _i64, _p, _p, _sz, _p]
 lib.gmla_gate_out.restype = _st
 lib.gmla_gate_out_workspace_size.argtypes = [_i64, _i64]
@@ -189,6 +194,26 @@ def gmla_attend_decode(Q, C, L, W_k, W_v, O, num_heads, scale=0.0, G=None, weigh
     code = lib.gmla_attend_decode(_ptr(Q), _ptr(C), B, Lmax, L, H, D, d_c, _ptr(W_k), _ptr(W_v), float(scale),
                                   _ptr(G), _ptr(O), _ptr(weights), wp, wb, _stream(stream))
     return _check(code, "gmla_attend_decode") if check else code
+
+
+def gmla_attend_decode_noalloc_max_bytes() -> int:
+    return lib.gmla_attend_decode_noalloc_max_bytes()
+
+
+def gmla_attend_decode_noalloc(Q, C, L, W_k, W_v, O, num_heads, scale=0.0, G=None, weights=None, stream=None,
+                               check=True):
+    """gmla_attend_decode without a workspace, for callers that cannot allocate device
+    memory at decode time; the scratch is a fixed array inside the library (see
+    include/gmla.h).  Calls that overlap on the GPU share that array and race."""
+    for n, t in (("Q", Q), ("C", C), ("W_k", W_k), ("W_v", W_v), ("O", O), ("G", G)):
+        _bf16(t, n)
+    B, d = Q.shape
+    H = int(num_heads)
+    D = d // H
+    _, Lmax, d_c = C.shape
+    code = lib.gmla_attend_decode_noalloc(_ptr(Q), _ptr(C), B, Lmax, L, H, D, d_c, _ptr(W_k), _ptr(W_v),
+                                          float(scale), _ptr(G), _ptr(O), _ptr(weights), _stream(stream))
+    return _check(code, "gmla_attend_decode_noalloc") if check else code
 
 
 def gmla_gate_out_workspace_size(M, d_model) -> int:

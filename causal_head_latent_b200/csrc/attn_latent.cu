@@ -11,6 +11,8 @@
 //            per split the running max m, sum l and acc[h,:] = sum_s p_s c_s
 //   combine  exact log-sum-exp merge of the splits, c^ = acc / l, then
 //            o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store.
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -166,17 +168,20 @@ void latent_plan(long long B, long long L, int *n_splits, int *keys_per_split) {
 
 // Workspace layout (each region 256-byte aligned):
 //   q~ bf16 [B,H,dc] | m, l float [S,B,H] each | acc float [S,B,H,dc] | lse2 float [B,H]
-size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc) {
-  int S, kps;
-  latent_plan(B, L, &S, &kps);
+static size_t latent_workspace_bytes_for(long long B, long long H, long long dc, long long S) {
   return align256(2 * B * H * dc) + 2 * align256(sizeof(float) * S * B * H) + align256(sizeof(float) * S * B * H * dc) +
          align256(sizeof(float) * B * H);
 }
 
-int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
-  using namespace latent;
+size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc) {
   int S, kps;
-  latent_plan(a.B, a.L, &S, &kps);
+  latent_plan(B, L, &S, &kps);
+  return latent_workspace_bytes_for(B, H, dc, S);
+}
+
+// The three launches for a given split plan (S splits of kps keys) and workspace.
+static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaStream_t stream) {
+  using namespace latent;
   uint8_t *ws = static_cast<uint8_t *>(a.workspace);
   uint16_t *qt = reinterpret_cast<uint16_t *>(ws);
   ws += align256(2 * (size_t)a.B * a.H * a.dc);
@@ -224,6 +229,71 @@ int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
   }
   if (a.weights) weights_fix_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, a.B * a.H, a.L);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
+  int S, kps;
+  latent_plan(a.B, a.L, &S, &kps);
+  return launch_attend_latent_plan(a, S, kps, stream);
+}
+
+// ------------------------------------------------------------------ decode without a caller workspace
+//
+// Some callers cannot allocate device memory when they decode: a runtime that
+// reserved all of the device memory for its own pool up front, or host code
+// that runs where the CUDA allocator must not be called (it can synchronise
+// the device, or the caller holds a lock the allocator may wait on).  For
+// them the decode scratch (q~, the per-split partial states and the
+// log-sum-exp) lives in the fixed array below, which every GPU that loads this
+// library holds until the process exits.
+//
+// Every call uses the same array and leaves its contents behind.  Each call
+// overwrites all of the scratch it reads before reading it (q~ by the absorb
+// kernel, every split's m, l and acc by the streaming kernel, the
+// log-sum-exp by the combine kernel), so nothing needs clearing.  Calls whose
+// GPU work overlaps -- on different streams, or from different host threads
+// without ordering -- race on the array.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+static constexpr int kNoAllocMaxDevices = 64;
+static void *g_decode_scratch_addr[kNoAllocMaxDevices];
+static std::mutex g_decode_scratch_mu;
+
+// Device address of the scratch array on the current device.  The symbol's
+// name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+static void *decode_scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_decode_scratch_mu);
+  if (!g_decode_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+    g_decode_scratch_addr[dev] = p;
+  }
+  return g_decode_scratch_addr[dev];
+}
+
+size_t latent_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Returns 0 on success, -1 on a CUDA error, -3 when the problem does not fit in
+// the scratch array even with a single split.  Allocates nothing.
+int launch_attend_latent_noalloc(const LatentArgs &args, cudaStream_t stream) {
+  int S, kps;
+  latent_plan(args.B, args.L, &S, &kps);
+  // fewer splits when the default plan's partial states do not fit
+  while (S > 1 && latent_workspace_bytes_for(args.B, args.H, args.dc, S) > kNoAllocScratchBytes) --S;
+  if (latent_workspace_bytes_for(args.B, args.H, args.dc, S) > kNoAllocScratchBytes) return -3;
+  const int KT = latent_tc_tile_keys();
+  const long long tiles = (args.L + KT - 1) / KT;
+  kps = (int)(((tiles + S - 1) / S) * KT);
+  S = (int)((args.L + kps - 1) / kps);  // no empty split
+  void *scratch = decode_scratch_address();
+  if (!scratch) return -1;
+  LatentArgs a = args;
+  a.workspace = scratch;
+  return launch_attend_latent_plan(a, S, kps, stream);
 }
 
 }  // namespace gmla

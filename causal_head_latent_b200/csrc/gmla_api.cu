@@ -316,6 +316,34 @@ gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B
   return launch_attend_latent(a, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ decode without a caller workspace
+
+size_t gmla_attend_decode_noalloc_max_bytes(void) { return latent_noalloc_scratch_bytes(); }
+
+gmla_status gmla_attend_decode_noalloc(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B, int64_t cache_len_max,
+                                       int64_t L, int64_t H, int64_t D_h, int64_t d_c, const gmla_bf16 *W_k,
+                                       const gmla_bf16 *W_v, float scale, const gmla_bf16 *G, gmla_bf16 *O,
+                                       float *weights, gmla_stream_t stream) {
+  if (!Q || !C || !W_k || !W_v || !O) return GMLA_ERR_ARG;
+  if (B <= 0 || H <= 0 || D_h <= 0 || d_c <= 0 || L < 1 || cache_len_max < L) return GMLA_ERR_ARG;
+  const void *ptrs[] = {Q, C, W_k, W_v, G, O};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (D_h != 128 || d_c % 64 != 0 || d_c > 512 || H > 96) return GMLA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || L > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D_h);
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  LatentArgs a{};
+  a.Q = Q; a.C = C; a.Wk = W_k; a.Wv = W_v; a.G = G; a.O = O; a.weights = weights;
+  a.cache_len_max = cache_len_max;
+  a.B = (int)B; a.L = (int)L; a.H = (int)H; a.dc = (int)d_c;
+  a.scale = scale; a.workspace = nullptr; a.status = st;
+  const int rc = launch_attend_latent_noalloc(a, static_cast<cudaStream_t>(stream));
+  if (rc == -3) return GMLA_ERR_WORKSPACE;
+  return rc == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ output projection
 
 size_t gmla_gate_out_workspace_size(int64_t M, int64_t d_model) {

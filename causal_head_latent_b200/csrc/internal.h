@@ -74,6 +74,10 @@ struct LatentArgs {
 };
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream);
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc);
+// Same launches with the scratch in a fixed device array of this library
+// (no workspace argument).  Returns 0, -1 (CUDA error) or -3 (too large).
+int launch_attend_latent_noalloc(const LatentArgs &a, cudaStream_t stream);
+size_t latent_noalloc_scratch_bytes();
 
 int num_sms();
 

@@ -160,6 +160,40 @@ GMLA_API gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, 
 GMLA_API size_t gmla_attend_decode_workspace_size(int64_t B, int64_t L, int64_t H, int64_t d_c);
 
 /*
+ * gmla_attend_decode_noalloc -- gmla_attend_decode for callers that cannot
+ * allocate device memory.  No page has a counterpart: it is a service of this
+ * library, not a step of the method.
+ *
+ * Some callers cannot hand over a workspace: a serving runtime that reserved
+ * all device memory for its own pool up front, or host code running where the
+ * CUDA allocator must not be called (the allocator can synchronise the device
+ * or wait on a lock the caller holds).  This entry point takes the same
+ * arguments as gmla_attend_decode minus the workspace and computes the same
+ * result (the key range may be split into fewer pieces, so float32 rounding
+ * may differ slightly).  Its scratch (q~, the per-split softmax states and the
+ * log-sum-exp) lives in one fixed device array of
+ * gmla_attend_decode_noalloc_max_bytes() bytes (32 MiB) inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *  - Allocates nothing and calls no allocating routine.
+ *  - Problems whose scratch does not fit even with a single key split
+ *    (about B*H*d_c*6 bytes > 32 MiB, e.g. B > 113 at H = 96, d_c = 512) return
+ *    GMLA_ERR_WORKSPACE before any launch.
+ *  - Every call shares the array and leaves its contents behind; each call
+ *    rewrites all the scratch it reads, so nothing needs clearing.  Calls whose
+ *    GPU work overlaps (different streams, or unordered host threads) race on
+ *    the array: order them on one stream.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current).
+ */
+GMLA_API gmla_status gmla_attend_decode_noalloc(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B,
+                                               int64_t cache_len_max, int64_t L, int64_t H, int64_t D_h,
+                                               int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v,
+                                               float scale, const gmla_bf16 *G, gmla_bf16 *O, float *weights,
+                                               gmla_stream_t stream);
+GMLA_API size_t gmla_attend_decode_noalloc_max_bytes(void);
+
+/*
  * gmla_gate_out -- the output projection Y = O W_o^T over M = B*T rows.
  * "Gated MLA" page, "The channel-wise output gate" (gate before W_o) and
  * step 6.  The gate is applied upstream (gmla_attend_prefill and
