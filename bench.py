@@ -67,6 +67,30 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
     return 2.0 * M * d * (2 * d + dc) + 2.0 * M * dc * 2 * d + prefill_flops(B, d // D, T) + 2.0 * M * d * d
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant kernels,
+# from one ncu capture each (profiles/).  Reported only while the kernel source is the one that
+# was captured (sha1 of the file); any change makes it null until the next capture.
+PROFILED_TRAFFIC = {
+    "attn_prefill.cu": {"sha1": "bb501558ebeb19bc821a219788ea5b8e5481a8d1", "bytes": 604.078848e6 + 185.454080e6,
+                        "how": "ncu capture at the timed size (B=1 H=96 T=8192)"},
+    "attn_latent_tc.cu": {"sha1": "c5244ae68f0d84b6ec11dcbad46f5d696cedb52e", "bytes": 640.111616e6 * 8 + 36.986112e6,
+                          "how": "ncu capture at L=16384, reads scaled x8 to L=131072 (cache traffic grows with L), "
+                                 "partial-state writes unscaled"},
+}
+
+
+def profiled_traffic(src):
+    import hashlib
+    ent = PROFILED_TRAFFIC.get(src)
+    path = os.path.join(ROOT, "causal_head_latent_b200", "csrc", src)
+    if not ent or not os.path.exists(path):
+        return None, None
+    with open(path, "rb") as f:
+        if hashlib.sha1(f.read()).hexdigest() != ent["sha1"]:
+            return None, "kernel changed since the ncu capture"
+    return ent["bytes"], ent["how"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -486,7 +510,10 @@ def main():
         line.update(value=val, unit="TFLOP/s")
         ach = pre.flops / (t_att / 1e3) / 1e12
         line["roofline"] = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"],
+                            "traffic": profiled_traffic("attn_prefill.cu")[0],
+                            "traffic_source": profiled_traffic("attn_prefill.cu")[1],
+                            "algorithmic_bytes": 2.0 * 4 * P_B * P_T * P_H * D,
                             "kernel": "attn_prefill_kernel",
                             "peak_kind": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)",
                             "frac_of_burst": ach / peaks["bf16_tflops"], "frac_of_datasheet_2250": ach / 2250.0}
@@ -496,7 +523,10 @@ def main():
         t_step = (perd["decode_project"] + perd["decode_attend"] + perd["decode_out"]) / K
         dobj = {"value": gbs * world, "unit": "GB/s", "ms_per_step": t_dec,
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "gmla_attend_decode",
+                             "frac": gbs / peaks["hbm_gbs"],
+                             "traffic": profiled_traffic("attn_latent_tc.cu")[0] if DEC_L == 131072 else None,
+                             "traffic_source": profiled_traffic("attn_latent_tc.cu")[1],
+                             "kernel": "gmla_attend_decode",
                              "peak_kind": f"{peaks['source']} HBM copy", "frac_of_datasheet_8000": gbs / 8000.0},
                 "step_ms": t_step, "step_gbs": decode_step_bytes() / (t_step / 1e3) / 1e9}
         line["decode"] = dobj
