@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict_
     float acc[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+#pragma unroll 8
     for (int d = 0; d < HD; ++d) {
       const float w = bf16_to_f32(Wk[((size_t)h * HD + d) * dc + c]);
 #pragma unroll
@@ -70,39 +71,51 @@ struct CombineParams {
   float *lse2;  // [B,H] log2-domain log-sum-exp (for the debug weights)
 };
 
-__global__ void __launch_bounds__(128) combine_kernel(const CombineParams P) {
-  extern __shared__ float chat[];  // [CB][dc]
+// grid (H, ceil(B / CB)), CT threads.  Per-split weights exp2(m_s - M) / L are
+// computed once per sequence; the merge runs over all (sequence, column) pairs;
+// two threads share one output row of W_v^(h) (one half of d_c each).
+constexpr int CT = 256;
+
+__global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
+  extern __shared__ float sm[];  // chat [CB][dc] | split weights [CB][n_splits]
   const int h = blockIdx.x, b0 = blockIdx.y * CB;
   const int nb = min(CB, P.B - b0);
-  const int dc = P.dc;
-  for (int bb = 0; bb < nb; ++bb) {
-    const int b = b0 + bb;
+  const int dc = P.dc, S = P.n_splits;
+  float *chat = sm;
+  float *wsp = sm + CB * dc;
+  if (threadIdx.x < nb) {
+    const int b = b0 + threadIdx.x;
     float M = -INFINITY;
-    for (int s = 0; s < P.n_splits; ++s) M = fmaxf(M, P.part_m[((size_t)s * P.B + b) * P.H + h]);
+    for (int s = 0; s < S; ++s) M = fmaxf(M, P.part_m[((size_t)s * P.B + b) * P.H + h]);
     float Lsum = 0.f;
-    for (int s = 0; s < P.n_splits; ++s) {
+    for (int s = 0; s < S; ++s) {
       const size_t i = ((size_t)s * P.B + b) * P.H + h;
-      if (P.part_m[i] != -INFINITY) Lsum += P.part_l[i] * fast_exp2(P.part_m[i] - M);
+      const float e = (P.part_m[i] == -INFINITY) ? 0.f : fast_exp2(P.part_m[i] - M);
+      wsp[threadIdx.x * S + s] = e;
+      Lsum += P.part_l[i] * e;
     }
     const float inv = 1.f / Lsum;
-    for (int c = threadIdx.x; c < dc; c += 128) {
-      float a = 0.f;
-      for (int s = 0; s < P.n_splits; ++s) {
-        const size_t i = ((size_t)s * P.B + b) * P.H + h;
-        const float ms = P.part_m[i];
-        if (ms != -INFINITY) a += P.part_acc[i * dc + c] * fast_exp2(ms - M);
-      }
-      chat[bb * dc + c] = a * inv;
-    }
-    if (threadIdx.x == 0 && P.lse2) P.lse2[(size_t)b * P.H + h] = M + __log2f(Lsum);
+    for (int s = 0; s < S; ++s) wsp[threadIdx.x * S + s] *= inv;
+    if (P.lse2) P.lse2[(size_t)b * P.H + h] = M + __log2f(Lsum);
   }
   __syncthreads();
-  const int i = threadIdx.x;
-  const uint16_t *w = P.Wv + ((size_t)h * HD + i) * dc;
+  for (int i = threadIdx.x; i < nb * dc; i += CT) {
+    const int bb = i / dc, c = i % dc;
+    const float *acc = P.part_acc + ((size_t)(b0 + bb) * P.H + h) * dc + c;
+    const size_t split_stride = (size_t)P.B * P.H * dc;
+    float a = 0.f;
+    for (int s = 0; s < S; ++s) a = fmaf(wsp[bb * S + s], acc[s * split_stride], a);
+    chat[i] = a;
+  }
+  __syncthreads();
+  const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
+  const int c_lo = half * (dc / 2), c_hi = c_lo + dc / 2;
+  const uint16_t *w = P.Wv + ((size_t)h * HD + r) * dc;
   float o[CB];
 #pragma unroll
   for (int bb = 0; bb < CB; ++bb) o[bb] = 0.f;
-  for (int c = 0; c < dc; c += 8) {
+#pragma unroll 4
+  for (int c = c_lo; c < c_hi; c += 8) {
     const uint4 v = *reinterpret_cast<const uint4 *>(w + c);
     const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -118,12 +131,16 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams P) {
     }
   }
 #pragma unroll
-  for (int bb = 0; bb < CB; ++bb) {
-    if (bb < nb) {
-      const size_t oi = (size_t)(b0 + bb) * P.H * HD + (size_t)h * HD + i;
-      float r = o[bb];
-      if (P.G) r *= sigmoidf_(bf16_to_f32(P.G[oi]));
-      P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+  for (int bb = 0; bb < CB; ++bb) o[bb] += __shfl_xor_sync(0xffffffffu, o[bb], 1);
+  if (half == 0) {
+#pragma unroll
+    for (int bb = 0; bb < CB; ++bb) {
+      if (bb < nb) {
+        const size_t oi = (size_t)(b0 + bb) * P.H * HD + (size_t)h * HD + r;
+        float v = o[bb];
+        if (P.G) v *= sigmoidf_(bf16_to_f32(P.G[oi]));
+        P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+      }
     }
   }
 }
@@ -225,7 +242,7 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     P.G = a.G;
     P.O = a.O;
     P.lse2 = lse2;
-    combine_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), 128, sizeof(float) * CB * a.dc, stream>>>(P);
+    combine_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), CT, sizeof(float) * (CB * a.dc + CB * S), stream>>>(P);
   }
   if (a.weights) weights_fix_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, a.B * a.H, a.L);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
