@@ -65,6 +65,8 @@ lib.gmla_gate_out_workspace_size.argtypes = [_i64, _i64]
 lib.gmla_gate_out_workspace_size.restype = _sz
 lib.gmla_get_device_status.argtypes = [_p]
 lib.gmla_get_device_status.restype = _st
+lib.gmla_selftest_wait_timeout.argtypes = [ctypes.c_uint, _p]
+lib.gmla_selftest_wait_timeout.restype = _st
 lib.gmla_status_string.argtypes = [_st]
 lib.gmla_status_string.restype = ctypes.c_char_p
 lib.gmla_version.argtypes = []
@@ -124,6 +126,11 @@ def gmla_version() -> int:
 def gmla_get_device_status(stream=None, raise_on_error: bool = True) -> int:
     code = lib.gmla_get_device_status(_stream(stream))
     return _check(code, "gmla_get_device_status") if raise_on_error else code
+
+
+def gmla_selftest_wait_timeout(milliseconds: int = 20, stream=None) -> int:
+    """Launch a kernel whose bounded wait runs out (see include/gmla.h); returns the launch status."""
+    return _check(lib.gmla_selftest_wait_timeout(int(milliseconds), _stream(stream)), "gmla_selftest_wait_timeout")
 
 
 def gmla_latent_project_workspace_size(B, T, d_model, d_c) -> int:

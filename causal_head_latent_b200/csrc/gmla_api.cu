@@ -10,6 +10,7 @@
 
 #include "../../include/gmla.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace gmla {
 
@@ -90,6 +91,18 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, int rank, const long long 
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// One thread waits, with a short bounded limit, on an mbarrier that nothing
+// arrives at: the wait runs out, records the timeout in the status word and the
+// kernel returns normally.
+__global__ void wait_timeout_kernel(unsigned *status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait_limit(&bar, 0, status, limit_ns);
+  }
+}
+
 }  // namespace gmla
 
 using namespace gmla;
@@ -123,6 +136,14 @@ gmla_status gmla_get_device_status(gmla_stream_t stream) {
   if (v & kStatusTimeout) return GMLA_ERR_TIMEOUT;
   if (v) return GMLA_ERR_CUDA;
   return GMLA_OK;
+}
+
+gmla_status gmla_selftest_wait_timeout(unsigned milliseconds, gmla_stream_t stream) {
+  if (milliseconds == 0 || milliseconds > 1000) return GMLA_ERR_ARG;
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(st, 1000000ull * milliseconds);
+  return cudaGetLastError() == cudaSuccess ? GMLA_OK : GMLA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ projections

@@ -212,6 +212,13 @@ GMLA_API size_t gmla_gate_out_workspace_size(int64_t M, int64_t d_model);
  * Returns GMLA_OK, GMLA_ERR_TIMEOUT (a bounded wait ran out) or GMLA_ERR_CUDA. */
 GMLA_API gmla_status gmla_get_device_status(gmla_stream_t stream);
 
+/* Self-test of the bounded-wait machinery (no counterpart on the pages): launches
+ * one thread that waits `milliseconds` (1..1000) on an mbarrier nothing arrives
+ * at; the wait runs out, records GMLA_ERR_TIMEOUT in the status word and the
+ * kernel returns.  A following gmla_get_device_status returns GMLA_ERR_TIMEOUT
+ * (and clears it); the CUDA context stays usable. */
+GMLA_API gmla_status gmla_selftest_wait_timeout(unsigned milliseconds, gmla_stream_t stream);
+
 /* Static, NUL-terminated description of a status code (host memory, never freed). */
 GMLA_API const char *gmla_status_string(gmla_status s);
 

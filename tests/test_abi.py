@@ -89,6 +89,12 @@ def test_host_validation_without_gpu(gmla):
     assert L.gmla_attend_decode(fake, fake, 2, 100, 100, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 16,
                                 None) == 5
     assert L.gmla_attend_decode_workspace_size(2, 100, 2, 64) > 16
+    # an empty query set is a no-op that launches nothing
+    assert L.gmla_attend_prefill(fake, s, fake, s, fake, s, 1, 2, 0, 300, 128, 1, 0.0, None, fake, s, None, None,
+                                 None) == 0
+    # the timeout self-test refuses limits outside 1..1000 ms
+    assert L.gmla_selftest_wait_timeout(0, None) == 1
+    assert L.gmla_selftest_wait_timeout(5000, None) == 1
     # gate_out: the gate is fused upstream
     assert L.gmla_gate_out(fake, fake, fake, 4, 256, fake, None, 0, None) == 2
     assert L.gmla_gate_out(None, None, fake, 4, 256, fake, None, 0, None) == 1
