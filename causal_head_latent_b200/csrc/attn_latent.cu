@@ -223,7 +223,9 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     const long long dq[3] = {a.dc, a.H, a.B}, sq[2] = {a.dc, (long long)a.H * a.dc};
     const unsigned bq[3] = {64, 96, 1};
     if (!make_tmap_bf16(&tq, qt, 3, dq, sq, bq)) return -1;
-    const long long dcm[3] = {a.dc, a.cache_len_max, a.B}, scm[2] = {a.dc, a.cache_len_max * a.dc};
+    // The key extent is L, not cache_len_max: rows of a ragged last tile past
+    // L read as zeros, never as whatever the unwritten cache rows hold.
+    const long long dcm[3] = {a.dc, a.L, a.B}, scm[2] = {a.dc, a.cache_len_max * a.dc};
     const unsigned bc[3] = {64, (unsigned)latent_tc_tile_keys(), 1};
     if (!make_tmap_bf16(&tc, a.C, 3, dcm, scm, bc)) return -1;
     if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, a.status, stream) != 0)
