@@ -3,39 +3,51 @@
 // One CTA streams the latents [k_begin, k_end) of one sequence b and keeps an
 // online-softmax state for all H (<= 96) heads at once; every latent tile is
 // read from HBM once and used twice, as keys and as values:
-//   S^T    [key, head]  = C_tile q~^T         M=64 keys, N=96 heads, K=d_c
-//   acc^T  [d_c, head] += C_tile^T P          M=128 per d_c block, N=96 heads,
-//                                             K=64 keys (C tile read MN-major)
-// with P [key, head] = 2^(S^T - m_head) held in shared memory as P^T rows.
-// q~ = scale*log2(e) * W_k^(h)T q_h comes from the absorb kernel (bfloat16),
-// so S is already in the exp2 domain.  P is rounded to bfloat16 before it
-// multiplies the latents, as in the eager attention path ("Kimi K3 - Softmax
-// over keys": float32 softmax, probabilities cast to the input type).
+//   S      [head, key]  = q~ C_tile^T          M=128 (heads, zero-padded by
+//                                               overlap), N=48 keys, K=d_c
+//   acc^T  [d_c, head] += C_tile^T P^T^T       M=128 per d_c block, N=96 heads,
+//                                               K=48 keys (C tile read MN-major)
+// with P^T [head, key] = 2^(S - m_head) in shared memory.  q~ = scale*log2(e) *
+// W_k^(h)T q_h comes from the absorb kernel (bfloat16), so S is already in
+// the exp2 domain.  P is rounded to bfloat16 before it multiplies the
+// latents, as in the eager attention path ("Kimi K3 - Softmax over keys":
+// float32 softmax, probabilities cast to the input type).
 //
-// Why keys on M: both products read their operands from shared memory, and on
-// sm_100a an MMA with a small N is bound by those reads (A + B bytes per
-// instruction), not by its arithmetic.  With keys on M, q~ is the 96-row B
-// operand (no padding to 128 rows) and one 64-key tile costs 32 score MMAs,
-// so the score product reads 2.5 KB of shared memory per key instead of the
-// 5 KB a heads-on-M, 32-key-tile product needs.
+// What bounds this kernel on sm_100a, and the shape that follows from it:
+//  * an SM takes in at most ~22.5 bytes per cycle through TMA, from L2 as
+//    from HBM, so the 1 KB latent row of a key costs >= 45 cycles of ingress
+//    and the latent stream has to stay in flight without gaps;
+//  * a tcgen05.mma with N <= 128 costs ~66 cycles whatever its M and N, so the
+//    MMA count per key sets the compute floor: 32 score + 12 value MMAs per
+//    48-key tile, ~61 cycles per key;
+//  * the MMA-issuing thread must not stall: a wait on its own recent MMAs
+//    (through a barrier and another warp) drains the MMA pipe, an acquire
+//    mbarrier wait between small MMAs costs ~270 cycles even when the phase
+//    has completed (a relaxed poll plus fence.acq_rel costs ~90), and each
+//    tcgen05.commit ~95.
+// Hence 48-key tiles: an 18-chunk latent ring (2.25 tiles) lets the loads of
+// tile j stream while tiles j-1 and j-2 are still in use; S is double-
+// buffered in TMEM so the score MMAs of the next tile never wait for the
+// softmax; the value MMAs of tile j-1 sit between the two parts of the score
+// MMAs of tile j, late enough for the softmax of tile j-1 and early enough
+// to release ring slots for tile j+2; and the ring moves in chunk pairs, so a
+// tile costs the MMA thread four data waits, one softmax wait and five
+// commits.
 //
-//   warp 0      TMA producer: q~ once, then the latent stream in 64-column
-//               chunks (8 KB: 64 keys x 64 d_c) through a 14-slot ring
+//   warp 0      TMA producer: q~ once, then the latents in 64-column chunks
+//               (6 KB: 48 keys x 64 d_c) through the ring
 //   warp 1      TMEM owner, MMA issuer (one thread)
-//   warps 2..5  softmax: each thread holds 2 keys x 24 heads of S^T; lazy
-//               rescale of acc^T when a head's running max grows by more than
-//               2^8; partial-state store
+//   warps 2..5  softmax, one head per TMEM lane; lazy rescale of acc^T when a
+//               head's running max grows by more than 2^8; partial-state store
 //
-// The ring holds 1.75 tiles, so the score MMAs of tile j are issued in two
-// parts around the value MMAs of tile j-1: the first six chunks of tile j
-// reuse slots tile j-2 released, the last two reuse the slots of chunks 0..1
-// of tile j-1, which the first d_c block of its value product releases.
-// Chunk pairs (2i, 2i+1) of a tile always sit in adjacent slots, so one
-// MN-major descriptor with a slot-sized leading offset spans a 128-row d_c
-// block.
+// q~ in shared memory: eight 64-column chunks of 96 rows (12 KB each) placed
+// 12 KB apart.  The score MMA reads 128-row A tiles, so rows 96..127 of chunk
+// k alias rows 0..31 of chunk k+1, and those of the last chunk the first 4 KB
+// of the P^T buffer that follows q~: they only feed S rows 96..127, which
+// nothing reads.
 //
-// TMEM columns: S^T [0, 96) in the M=64 layout (rows 16r..16r+15 in lanes
-// 32r..32r+15), acc^T blocks at 128 + 96*blk.
+// TMEM columns: S buffers at 0 and 64 (48 columns each), acc^T blocks at
+// 128 + 96*blk.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -43,22 +55,32 @@ namespace gmla {
 namespace latent_tc {
 
 constexpr int HMAX = 96;
-constexpr int KT = 64;                    // keys per tile: M of the score product
+constexpr int KT = 48;                    // keys per tile: N of the score product
 constexpr int NUM_THREADS = 192;
 constexpr int NCHUNK = 8;                 // 64-wide d_c chunks per tile (d_c <= 512)
 constexpr int QCHUNK = HMAX * 128;        // 12 KB: one d_c chunk of q~ for 96 heads
 constexpr int Q_BYTES = NCHUNK * QCHUNK;  // 96 KB
-constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row of 64 keys per head
-constexpr int CCHUNK = KT * 128;          // 8 KB: one d_c chunk of a 64-key tile
-constexpr int NSLOT = 14;                 // latent ring depth in chunks
-constexpr int NEARLY = NSLOT - NCHUNK;    // score chunks issued before the previous tile's value product
+constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row (48 keys used) per head
+constexpr int CCHUNK = KT * 128;          // 6 KB: one d_c chunk of a 48-key tile
+constexpr int NSLOT = 18;                 // latent ring depth in chunks
+constexpr int NPAIR = NSLOT / 2;          // the ring moves in chunk pairs (one 128-row d_c block)
+constexpr int NEARLY_PAIRS = 3;           // score chunk pairs of tile j issued before the value MMAs of tile j-1
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int kPrefetchTiles = 8;         // L2 prefetch distance of the latent stream
-constexpr int TM_S = 0;
-constexpr int TM_ACC = 128;
+constexpr int kPrefetchTiles = 3;         // L2 prefetch distance of the latent stream
+constexpr int TM_S = 0;                   // S buffers at TM_S + 64*i
+constexpr int TM_ACC = 128;               // acc^T blocks: 128 + 96*blk
 constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-path drain of copies / MMAs
 
-static_assert(NSLOT % 2 == 0 && NEARLY >= 2 && NEARLY <= NCHUNK, "ring depth");
+// Ring reuse: the chunks move in pairs (2i, 2i+1) -- the two halves of d_c
+// block i -- through NPAIR pair slots with one full and one empty barrier
+// each, so the MMA thread waits once per 8 score MMAs and releases a pair
+// with one commit per value block.  Pair q of tile j sits in pair slot
+// (4j + q) % NPAIR; its previous user belongs to tile j-2 or earlier, whose
+// value MMAs were issued an iteration before the score MMAs that need the
+// slot.  The two chunks of a pair are adjacent, so one MN-major descriptor
+// with a chunk-sized leading offset spans the 128-row d_c block.
+static_assert(NSLOT % 2 == 0 && NPAIR >= 2 * (NCHUNK / 2) + 1, "ring depth");
+static_assert(P_BYTES >= 32 * 128, "P^T buffer must cover the q~ tail");
 
 struct Params {
   const uint16_t *C;  // latent cache [B, Lmax, dc] (for the L2 prefetch stream)
@@ -69,16 +91,13 @@ struct Params {
   unsigned *status;
 };
 
-// 96 float32 columns of an M=64 accumulator in the 16x256b shape: this warp's
-// 16 rows (lanes 32r..32r+15), thread t gets rows t/4 and t/4+8, column pair
-// 2*(t%4) of every 8-column group.  v[4i + 2a + e] = (row t/4 + 8a, column
-// 8i + 2*(t%4) + e).
-__device__ __forceinline__ void tmem_ld_m64_96(uint32_t taddr, float *v) {
+// 48 consecutive float32 columns of this thread's TMEM lane (warp-wide).
+__device__ __forceinline__ void tmem_ld48(uint32_t taddr, float *v) {
   uint32_t r[48];
   asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
       "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%48];\n\t"
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47}, "
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47}, "
       "[%49];\n\t"
       "tcgen05.wait::ld.sync.aligned;\n"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
@@ -87,7 +106,7 @@ __device__ __forceinline__ void tmem_ld_m64_96(uint32_t taddr, float *v) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]),
         "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]),
         "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47])
-      : "r"(taddr), "r"(taddr + 64)
+      : "r"(taddr), "r"(taddr + 32)
       : "memory");
 #pragma unroll
   for (int i = 0; i < 48; ++i) v[i] = __uint_as_float(r[i]);
@@ -108,28 +127,21 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Byte offset of P^T[h][key] in the 128-byte-swizzled K-major P^T buffer.
-__device__ __forceinline__ uint32_t pt_offset(int h, int key) {
-  return (uint32_t)(h * 128 + ((((key >> 3) ^ (h & 7)) << 4) | ((key & 7) << 1)));
-}
-
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     latent_decode_kernel(const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmC,
                          const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sq = base;
-  uint8_t *sp = sq + Q_BYTES;
+  uint8_t *sp = sq + Q_BYTES;  // directly after q~: it holds the padded rows' tail
   uint8_t *sc = sp + P_BYTES;  // Q_BYTES + P_BYTES is a multiple of 1024
   float *alpha_s = reinterpret_cast<float *>(sc + NSLOT * CCHUNK);
-  float *red_s = alpha_s + 128;  // [4][HMAX]: per-quarter partial max / sum
-  uint64_t *bars = reinterpret_cast<uint64_t *>(red_s + 4 * HMAX);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(alpha_s + 128);
   uint64_t *bar_q = bars;
-  uint64_t *c_full = bars + 1;           // [NSLOT]
-  uint64_t *c_empty = c_full + NSLOT;    // [NSLOT]
-  uint64_t *s_full = c_empty + NSLOT;
-  uint64_t *s_free = s_full + 1;
-  uint64_t *p_full = s_free + 1;
+  uint64_t *c_full = bars + 1;           // [NPAIR]
+  uint64_t *c_empty = c_full + NPAIR;    // [NPAIR]
+  uint64_t *s_full = c_empty + NPAIR;    // [2]
+  uint64_t *p_full = s_full + 2;
   uint64_t *acc_done = p_full + 1;
   uint64_t *mma_idle = acc_done + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_idle + 1);
@@ -143,12 +155,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < NSLOT; ++s) {
+    for (int s = 0; s < NPAIR; ++s) {
       mbar_init(&c_full[s], 1);
       mbar_init(&c_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
+    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(p_full, 4);
     mbar_init(acc_done, 1);
     mbar_init(mma_idle, 1);
@@ -169,9 +180,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tmC);
       mbar_arrive_expect_tx(bar_q, Q_BYTES);
       for (int kc = 0; kc < NCHUNK; ++kc) tma_load_3d(sq + kc * QCHUNK, &tmQt, bar_q, kc * 64, 0, b);
-      // The latents of this split are one contiguous range; an L2 prefetch
-      // stream kPrefetchTiles ahead of the ring hides DRAM latency without
-      // more shared memory.
+      // The latents of this split are one contiguous range; a short L2
+      // prefetch stream ahead of the ring starts the DRAM reads early.
       const uint8_t *crow = reinterpret_cast<const uint8_t *>(p.C + ((size_t)b * p.Lmax) * p.dc);
       const size_t key_bytes = (size_t)p.dc * 2;
       auto prefetch_tile = [&](int jt) {
@@ -179,67 +189,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (jt < n_tiles) prefetch_l2_bulk(crow + (size_t)kb * key_bytes, (uint32_t)(min(KT, k_end - kb) * key_bytes));
       };
       for (int jt = 1; jt < kPrefetchTiles; ++jt) prefetch_tile(jt);
-      const int n_chunks = n_tiles * NCHUNK;
+      const int n_pairs = n_tiles * (NCHUNK / 2);
       int issued = 0;
-      for (int g = 0; g < n_chunks; ++g) {
-        const int s = g % NSLOT, use = g / NSLOT, j = g / NCHUNK, kc = g % NCHUNK;
-        if (kc == 0) prefetch_tile(j + kPrefetchTiles);
-        if (!mbar_wait(&c_empty[s], (use & 1) ^ 1, p.status)) break;
-        mbar_arrive_expect_tx(&c_full[s], CCHUNK);
-        tma_load_3d(sc + s * CCHUNK, &tmC, &c_full[s], kc * 64, k_begin + j * KT, b);
+      for (int g = 0; g < n_pairs; ++g) {
+        const int ps = g % NPAIR, use = g / NPAIR, j = g / (NCHUNK / 2), q = g % (NCHUNK / 2);
+        if (q == 0) prefetch_tile(j + kPrefetchTiles);
+        if (!mbar_wait_relaxed(&c_empty[ps], (use & 1) ^ 1, p.status)) break;
+        mbar_arrive_expect_tx(&c_full[ps], 2 * CCHUNK);
+        for (int h2 = 0; h2 < 2; ++h2)
+          tma_load_3d(sc + (2 * ps + h2) * CCHUNK, &tmC, &c_full[ps], (2 * q + h2) * 64, k_begin + j * KT, b);
         issued = g + 1;
       }
       // Error path: let the copies still in flight land before the CTA exits.
-      if (issued < n_chunks)
-        for (int g = max(0, issued - NSLOT); g < issued; ++g)
-          mbar_wait_limit(&c_full[g % NSLOT], (g / NSLOT) & 1, p.status, kDrainLimitNs);
+      if (issued < n_pairs)
+        for (int g = max(0, issued - NPAIR); g < issued; ++g)
+          mbar_wait_limit(&c_full[g % NPAIR], (g / NPAIR) & 1, p.status, kDrainLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(KT, HMAX, false, false);
+      constexpr uint32_t idS = idesc_bf16_f32(128, KT, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, HMAX, true, false);
       const uint32_t aq = smem_u32(sq), ac = smem_u32(sc), ap = smem_u32(sp);
-      auto score_chunks = [&](int j, int kc0, int kc1) -> bool {
-        for (int kc = kc0; kc < kc1; ++kc) {
-          const int g = j * NCHUNK + kc;
+      // Score MMAs of chunk pairs [q0, q1) of tile j into S buffer j&1.  That
+      // buffer was last read by the softmax of tile j-2, whose p_full this
+      // thread waited for (followed by tcgen05.fence::after_thread_sync)
+      // before the value MMAs of tile j-2.
+      auto score_pairs = [&](int j, int q0, int q1) -> bool {
+        const uint32_t dS = tmem + TM_S + (j & 1) * 64;
+        for (int q = q0; q < q1; ++q) {
+          const int g = j * (NCHUNK / 2) + q;
           // TMA completion on the mbarrier orders the copy before the MMA's reads
-          if (!mbar_wait(&c_full[g % NSLOT], (g / NSLOT) & 1, p.status)) return false;
-          const uint32_t cst = ac + (g % NSLOT) * CCHUNK;
+          if (!mbar_wait_relaxed(&c_full[g % NPAIR], (g / NPAIR) & 1, p.status)) return false;
+          const uint32_t cst = ac + (g % NPAIR) * 2 * CCHUNK;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ss(tmem + TM_S, sdesc_sw128(cst + kk * 32, 16, 1024),
-                         sdesc_sw128(aq + kc * QCHUNK + kk * 32, 16, 1024), idS, (kc | kk) ? 1u : 0u);
+          for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(dS, sdesc_sw128(aq + (2 * q + h2) * QCHUNK + kk * 32, 16, 1024),
+                           sdesc_sw128(cst + h2 * CCHUNK + kk * 32, 16, 1024), idS, (q | h2 | kk) ? 1u : 0u);
         }
         return true;
       };
       bool ok = mbar_wait(bar_q, 0, p.status);
       for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          // S^T is single-buffered: the softmax must have read S^T_{j-1}.
-          if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1, p.status)) break;
-          tc_fence_after();
-          if (!score_chunks(j, 0, NEARLY)) break;
-        }
+        if (j < n_tiles && !score_pairs(j, 0, NEARLY_PAIRS)) break;
         if (j >= 1) {
           const int jp = j - 1;
-          if (!mbar_wait(p_full, jp & 1, p.status)) break;
+          if (!mbar_wait_relaxed(p_full, jp & 1, p.status)) break;
           tc_fence_after();
 #pragma unroll
           for (int blk = 0; blk < 4; ++blk) {
-            const int g0 = jp * NCHUNK + 2 * blk;  // even, so g0 % NSLOT and the next slot are adjacent
-            const uint32_t cst = ac + (g0 % NSLOT) * CCHUNK;
+            const int g = jp * (NCHUNK / 2) + blk;
+            const uint32_t cst = ac + (g % NPAIR) * 2 * CCHUNK;
 #pragma unroll
             for (int ks = 0; ks < KT / 16; ++ks)
               umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
                            sdesc_sw128(ap + ks * 32, 16, 1024), idPV, (jp > 0 || ks > 0) ? 1u : 0u);
-            umma_commit(&c_empty[g0 % NSLOT]);
-            umma_commit(&c_empty[(g0 + 1) % NSLOT]);
+            umma_commit(&c_empty[g % NPAIR]);
           }
           if (jp == n_tiles - 1) umma_commit(acc_done);
         }
         if (j < n_tiles) {
-          if (!score_chunks(j, NEARLY, NCHUNK)) break;
-          umma_commit(s_full);  // also orders P^T and acc^T after the value MMAs of tile j-1
+          if (!score_pairs(j, NEARLY_PAIRS, NCHUNK / 2)) break;
+          // Arrives once S_j and everything issued before it -- the value
+          // MMAs of tile j-1 among them -- have completed, so the softmax of
+          // tile j may rewrite P^T and rescale acc^T.
+          umma_commit(&s_full[j & 1]);
         }
       }
       // Every path: wait until the MMAs issued so far have finished before
@@ -249,88 +264,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int h = quarter * 32 + lane;  // head owned in the S phase; d_c row in the acc phase
+    const bool head_ok = h < p.H;
+    const bool active = quarter < 3;  // lanes 96..127 of S hold only padding rows
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int r8 = lane >> 2, c4 = lane & 3;
-    const int keyA = 16 * quarter + r8;  // tile rows of v[4i + e] (keyA) and v[4i + 2 + e] (keyA + 8)
-    float m[24], ls[24];
-#pragma unroll
-    for (int k = 0; k < 24; ++k) {
-      m[k] = -INFINITY;
-      ls[k] = 0.f;
-    }
-    float *wbase = p.weights ? p.weights + (size_t)b * p.H * (size_t)p.L : nullptr;
+    float m_used = -INFINITY, l = 0.f;
+    uint8_t *prow = sp + h * 128;
+    const int sw = h & 7;
+    float *wrow = (p.weights && head_ok) ? p.weights + ((size_t)b * p.H + h) * (size_t)p.L : nullptr;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const bool got = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, p.status));
-      float v[48];
+      const int sb = j & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait_relaxed(&s_full[sb], (j >> 1) & 1, p.status));
+      float x[KT];
       if (got) {
         tc_fence_after();
-        tmem_ld_m64_96(tmem + lane_off + TM_S, v);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (active) {
+          tmem_ld48(tmem + lane_off + TM_S + sb * 64, x);
+        } else {
+#pragma unroll
+          for (int c = 0; c < KT; ++c) x[c] = -INFINITY;
+        }
       }
       const int k0 = k_begin + j * KT;
-      const bool okA = got && k0 + keyA < k_end, okB = got && k0 + keyA + 8 < k_end;
-      float mx[24];
-      bool need = !got;
+      float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 12; ++i)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float a = okA ? v[4 * i + e] : -INFINITY;
-          const float c = okB ? v[4 * i + 2 + e] : -INFINITY;
-          v[4 * i + e] = a;
-          v[4 * i + 2 + e] = c;
-          mx[2 * i + e] = fmaxf(a, c);
-          need |= mx[2 * i + e] > m[2 * i + e] + kRescaleThreshold;
-        }
-      if (wbase) {
-#pragma unroll
-        for (int i = 0; i < 12; ++i)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = 8 * i + 2 * c4 + e;
-            if (h < p.H) {
-              float *w = wbase + (size_t)h * p.L + k0 + keyA;
-              if (okA) w[0] = v[4 * i + e];
-              if (okB) w[8] = v[4 * i + 2 + e];
-            }
-          }
+      for (int c = 0; c < KT; ++c) {
+        if (!got || k0 + c >= k_end) x[c] = -INFINITY;
+        mx = fmaxf(mx, x[c]);
       }
-      if (bar_or(1, 128, need)) {
+      if (wrow) {
+#pragma unroll
+        for (int c = 0; c < KT; ++c)
+          if (k0 + c < k_end) wrow[k0 + c] = x[c];
+      }
+      const bool need = head_ok && mx > m_used + kRescaleThreshold;
+      if (bar_or(1, 128, need || !got)) {
         if (bar_or(1, 128, !got)) {  // a wait gave up: every softmax thread leaves together
           ok = false;
           break;
         }
-        // exact tile max per head: over the 8 threads sharing c4, then over the quarters
-#pragma unroll
-        for (int k = 0; k < 24; ++k) {
-          mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 4));
-          mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 8));
-          mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 16));
+        float alpha = 1.f;
+        if (need) {
+          if (m_used != -INFINITY) alpha = fast_exp2(m_used - mx);
+          m_used = mx;
         }
-        if (r8 == 0) {
-#pragma unroll
-          for (int i = 0; i < 12; ++i)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) red_s[quarter * HMAX + 8 * i + 2 * c4 + e] = mx[2 * i + e];
-        }
-        bar_sync(1, 128);
-#pragma unroll
-        for (int i = 0; i < 12; ++i)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = 8 * i + 2 * c4 + e, k = 2 * i + e;
-            const float tm = fmaxf(fmaxf(red_s[h], red_s[HMAX + h]), fmaxf(red_s[2 * HMAX + h], red_s[3 * HMAX + h]));
-            float alpha = 1.f;
-            if (tm > m[k] + kRescaleThreshold) {
-              if (m[k] != -INFINITY) alpha = fast_exp2(m[k] - tm);
-              m[k] = tm;
-            }
-            ls[k] *= alpha;
-            if (quarter == 0 && r8 == 0) alpha_s[h] = alpha;
-          }
+        l *= alpha;
+        alpha_s[h] = alpha;
         bar_sync(1, 128);  // alpha_s complete
         if (j > 0) {
           // acc^T lanes are d_c rows, columns are heads: scale column h by
@@ -348,21 +328,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        bar_sync(1, 128);  // red_s and alpha_s are rewritten by a later tile
+        bar_sync(1, 128);  // alpha_s is rewritten by a later tile
       }
-      // probabilities, rounded to bfloat16 into P^T (free: the value MMAs of
-      // tile j-1 completed before s_full of tile j)
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      float rs = 0.f;
+      uint32_t pk[KT / 2];
 #pragma unroll
-      for (int i = 0; i < 12; ++i)
+      for (int c = 0; c < KT; c += 2) {
+        const float p0 = fast_exp2(x[c] - mref), p1 = fast_exp2(x[c + 1] - mref);
+        rs += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l += rs;
+      // P^T row h (free: the value MMAs of tile j-1 completed before s_full)
+      if (active) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = 8 * i + 2 * c4 + e, k = 2 * i + e;
-          const float mref = (m[k] == -INFINITY) ? 0.f : m[k];
-          const float pa = fast_exp2(v[4 * i + e] - mref), pb = fast_exp2(v[4 * i + 2 + e] - mref);
-          ls[k] += pa + pb;
-          *reinterpret_cast<uint16_t *>(sp + pt_offset(h, keyA)) = __bfloat16_as_ushort(__float2bfloat16_rn(pa));
-          *reinterpret_cast<uint16_t *>(sp + pt_offset(h, keyA + 8)) = __bfloat16_as_ushort(__float2bfloat16_rn(pb));
-        }
+        for (int u = 0; u < KT / 8; ++u)
+          *reinterpret_cast<uint4 *>(prow + ((u ^ sw) << 4)) =
+              make_uint4(pk[u * 4 + 0], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -374,31 +358,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool fin = !bar_or(1, 128, !mbar_wait(acc_done, 0, p.status));
       if (fin) {
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 24; ++k) {
-          ls[k] += __shfl_xor_sync(0xffffffffu, ls[k], 4);
-          ls[k] += __shfl_xor_sync(0xffffffffu, ls[k], 8);
-          ls[k] += __shfl_xor_sync(0xffffffffu, ls[k], 16);
-        }
-        if (r8 == 0) {
-#pragma unroll
-          for (int i = 0; i < 12; ++i)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) red_s[quarter * HMAX + 8 * i + 2 * c4 + e] = ls[2 * i + e];
-        }
-        bar_sync(1, 128);
         const size_t rec = ((size_t)split * p.B + b) * p.H;
-        if (quarter == 0 && r8 == 0) {
-#pragma unroll
-          for (int i = 0; i < 12; ++i)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int h = 8 * i + 2 * c4 + e;
-              if (h < p.H) {
-                p.part_m[rec + h] = m[2 * i + e];
-                p.part_l[rec + h] = (red_s[h] + red_s[HMAX + h]) + (red_s[2 * HMAX + h] + red_s[3 * HMAX + h]);
-              }
-            }
+        if (head_ok) {
+          p.part_m[rec + h] = m_used;
+          p.part_l[rec + h] = l;
         }
         const int row = quarter * 32 + lane;  // d_c row within a block
 #pragma unroll 1
@@ -429,7 +392,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 size_t smem_bytes() {
-  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 4 * HMAX * 4 + 8 * (1 + 2 * NSLOT + 5) + 16;
+  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 2 * NPAIR + 5) + 16;
 }
 
 }  // namespace latent_tc
