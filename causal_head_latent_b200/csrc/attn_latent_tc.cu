@@ -31,7 +31,7 @@
 // softmax; the value MMAs of tile j-1 sit between the two parts of the score
 // MMAs of tile j, late enough for the softmax of tile j-1 and early enough
 // to release ring slots for tile j+2; and the ring moves in chunk pairs, so a
-// tile costs the MMA thread four data waits, one softmax wait and five
+// tile costs the MMA thread two data waits, one softmax wait and three
 // commits.
 //
 //   warp 0      TMA producer: q~ once, then the latents in 64-column chunks
@@ -64,7 +64,9 @@ constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row (48 
 constexpr int CCHUNK = KT * 128;          // 6 KB: one d_c chunk of a 48-key tile
 constexpr int NSLOT = 18;                 // latent ring depth in chunks
 constexpr int NPAIR = NSLOT / 2;          // the ring moves in chunk pairs (one 128-row d_c block)
+constexpr int NPT = NCHUNK / 2;           // chunk pairs per tile
 constexpr int NEARLY_PAIRS = 3;           // score chunk pairs of tile j issued before the value MMAs of tile j-1
+constexpr int NTB = 4;                    // tile-indexed barriers rotate over 4 tiles
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kPrefetchTiles = 3;         // L2 prefetch distance of the latent stream
 constexpr int TM_S = 0;                   // S buffers at TM_S + 64*i
@@ -72,14 +74,21 @@ constexpr int TM_ACC = 128;               // acc^T blocks: 128 + 96*blk
 constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-path drain of copies / MMAs
 
 // Ring reuse: the chunks move in pairs (2i, 2i+1) -- the two halves of d_c
-// block i -- through NPAIR pair slots with one full and one empty barrier
-// each, so the MMA thread waits once per 8 score MMAs and releases a pair
-// with one commit per value block.  Pair q of tile j sits in pair slot
+// block i -- through NPAIR pair slots.  Pair q of tile j sits in pair slot
 // (4j + q) % NPAIR; its previous user belongs to tile j-2 or earlier, whose
 // value MMAs were issued an iteration before the score MMAs that need the
 // slot.  The two chunks of a pair are adjacent, so one MN-major descriptor
 // with a chunk-sized leading offset spans the 128-row d_c block.
-static_assert(NSLOT % 2 == 0 && NPAIR >= 2 * (NCHUNK / 2) + 1, "ring depth");
+//
+// Barriers are per tile (rotating over NTB tiles), not per slot, so that a
+// tile costs the MMA thread two data waits (pairs 0..2, pair 3) and two
+// release commits (pairs 0..1 after value blocks 0..1, pairs 2..3 after
+// blocks 2..3).  A rotating barrier is never more than one phase away from
+// the phase its waiter wants: the producer arms tile j only after the
+// release of tile j-2 or j-3, by which time the MMA thread has consumed
+// tile j-NTB; the producer waits for the release of tile j-2 or j-3 only
+// after it observed the releases of tiles j-4 and earlier.
+static_assert(NSLOT % 2 == 0 && NPAIR >= 2 * NPT + 1, "ring depth");
 static_assert(P_BYTES >= 32 * 128, "P^T buffer must cover the q~ tail");
 
 struct Params {
@@ -138,9 +147,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   float *alpha_s = reinterpret_cast<float *>(sc + NSLOT * CCHUNK);
   uint64_t *bars = reinterpret_cast<uint64_t *>(alpha_s + 128);
   uint64_t *bar_q = bars;
-  uint64_t *c_full = bars + 1;           // [NPAIR]
-  uint64_t *c_empty = c_full + NPAIR;    // [NPAIR]
-  uint64_t *s_full = c_empty + NPAIR;    // [2]
+  uint64_t *full_e = bars + 1;           // [NTB]: pairs 0..NEARLY_PAIRS-1 of tile j landed
+  uint64_t *full_l = full_e + NTB;       // [NTB]: the remaining pairs of tile j landed
+  uint64_t *rel = full_l + NTB;          // [NTB][2]: pairs 2h, 2h+1 of tile j released
+  uint64_t *s_full = rel + 2 * NTB;      // [2]
   uint64_t *p_full = s_full + 2;
   uint64_t *acc_done = p_full + 1;
   uint64_t *mma_idle = acc_done + 1;
@@ -155,9 +165,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < NPAIR; ++s) {
-      mbar_init(&c_full[s], 1);
-      mbar_init(&c_empty[s], 1);
+    for (int t = 0; t < NTB; ++t) {
+      mbar_init(&full_e[t], NEARLY_PAIRS);
+      mbar_init(&full_l[t], NPT - NEARLY_PAIRS);
+      mbar_init(&rel[2 * t], 1);
+      mbar_init(&rel[2 * t + 1], 1);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(p_full, 4);
@@ -189,21 +201,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (jt < n_tiles) prefetch_l2_bulk(crow + (size_t)kb * key_bytes, (uint32_t)(min(KT, k_end - kb) * key_bytes));
       };
       for (int jt = 1; jt < kPrefetchTiles; ++jt) prefetch_tile(jt);
-      const int n_pairs = n_tiles * (NCHUNK / 2);
+      const int n_pairs = n_tiles * NPT;
       int issued = 0;
       for (int g = 0; g < n_pairs; ++g) {
-        const int ps = g % NPAIR, use = g / NPAIR, j = g / (NCHUNK / 2), q = g % (NCHUNK / 2);
+        const int ps = g % NPAIR, j = g / NPT, q = g % NPT;
         if (q == 0) prefetch_tile(j + kPrefetchTiles);
-        if (!mbar_wait_relaxed(&c_empty[ps], (use & 1) ^ 1, p.status)) break;
-        mbar_arrive_expect_tx(&c_full[ps], 2 * CCHUNK);
+        if (g >= NPAIR) {  // the slot's previous pair: tile t, released with its half q' / 2
+          const int gp = g - NPAIR, t = gp / NPT, hq = (gp % NPT) / 2;
+          if (!mbar_wait_relaxed(&rel[2 * (t % NTB) + hq], (t / NTB) & 1, p.status)) break;
+        }
+        uint64_t *fb = q < NEARLY_PAIRS ? &full_e[j % NTB] : &full_l[j % NTB];
+        mbar_arrive_expect_tx(fb, 2 * CCHUNK);
         for (int h2 = 0; h2 < 2; ++h2)
-          tma_load_3d(sc + (2 * ps + h2) * CCHUNK, &tmC, &c_full[ps], (2 * q + h2) * 64, k_begin + j * KT, b);
+          tma_load_3d(sc + (2 * ps + h2) * CCHUNK, &tmC, fb, (2 * q + h2) * 64, k_begin + j * KT, b);
         issued = g + 1;
       }
-      // Error path: let the copies still in flight land before the CTA exits.
+      // Error path: let the copies still in flight land before the CTA exits
+      // (the tiles whose loads were issued and not consumed: at most 3).
       if (issued < n_pairs)
-        for (int g = max(0, issued - NPAIR); g < issued; ++g)
-          mbar_wait_limit(&c_full[g % NPAIR], (g / NPAIR) & 1, p.status, kDrainLimitNs);
+        for (int j = max(0, (issued - NPAIR) / NPT); j * NPT < issued; ++j) {
+          mbar_wait_limit(&full_e[j % NTB], (j / NTB) & 1, p.status, kDrainLimitNs);
+          if ((j + 1) * NPT <= issued) mbar_wait_limit(&full_l[j % NTB], (j / NTB) & 1, p.status, kDrainLimitNs);
+        }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -216,10 +235,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // before the value MMAs of tile j-2.
       auto score_pairs = [&](int j, int q0, int q1) -> bool {
         const uint32_t dS = tmem + TM_S + (j & 1) * 64;
+        // TMA completion on the mbarrier orders the copies before the MMA's reads
+        if (!mbar_wait_relaxed(q0 == 0 ? &full_e[j % NTB] : &full_l[j % NTB], (j / NTB) & 1, p.status)) return false;
         for (int q = q0; q < q1; ++q) {
-          const int g = j * (NCHUNK / 2) + q;
-          // TMA completion on the mbarrier orders the copy before the MMA's reads
-          if (!mbar_wait_relaxed(&c_full[g % NPAIR], (g / NPAIR) & 1, p.status)) return false;
+          const int g = j * NPT + q;
           const uint32_t cst = ac + (g % NPAIR) * 2 * CCHUNK;
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2)
@@ -239,18 +258,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int blk = 0; blk < 4; ++blk) {
-            const int g = jp * (NCHUNK / 2) + blk;
+            const int g = jp * NPT + blk;
             const uint32_t cst = ac + (g % NPAIR) * 2 * CCHUNK;
 #pragma unroll
             for (int ks = 0; ks < KT / 16; ++ks)
               umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
                            sdesc_sw128(ap + ks * 32, 16, 1024), idPV, (jp > 0 || ks > 0) ? 1u : 0u);
-            umma_commit(&c_empty[g % NPAIR]);
+            if (blk & 1) umma_commit(&rel[2 * (jp % NTB) + (blk >> 1)]);
           }
           if (jp == n_tiles - 1) umma_commit(acc_done);
         }
         if (j < n_tiles) {
-          if (!score_pairs(j, NEARLY_PAIRS, NCHUNK / 2)) break;
+          if (!score_pairs(j, NEARLY_PAIRS, NPT)) break;
           // Arrives once S_j and everything issued before it -- the value
           // MMAs of tile j-1 among them -- have completed, so the softmax of
           // tile j may rewrite P^T and rescale acc^T.
@@ -392,7 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 size_t smem_bytes() {
-  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 2 * NPAIR + 5) + 16;
+  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 4 * NTB + 5) + 16;
 }
 
 }  // namespace latent_tc
