@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (q == 0) prefetch_tile(j + kPrefetchTiles);
         if (g >= NPAIR) {  // the slot's previous pair: tile t, released with its half q' / 2
           const int gp = g - NPAIR, t = gp / NPT, hq = (gp % NPT) / 2;
-          if (!mbar_wait_relaxed(&rel[2 * (t % NTB) + hq], (t / NTB) & 1, p.status)) break;
+          if (!mbar_wait(&rel[2 * (t % NTB) + hq], (t / NTB) & 1, p.status)) break;
         }
         uint64_t *fb = q < NEARLY_PAIRS ? &full_e[j % NTB] : &full_l[j % NTB];
         mbar_arrive_expect_tx(fb, 2 * CCHUNK);
@@ -294,7 +294,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int sb = j & 1;
-      const bool got = __all_sync(0xffffffffu, mbar_wait_relaxed(&s_full[sb], (j >> 1) & 1, p.status));
+      // a suspending wait: polling warps would take shared-memory bandwidth from the MMAs
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1, p.status));
       float x[KT];
       if (got) {
         tc_fence_after();

@@ -79,10 +79,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
   }
 }
 
-__device__ __forceinline__ bool mbar_test_wait_relaxed(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait_relaxed(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred P;\n\tmbarrier.test_wait.parity.relaxed.cta.shared::cta.b64 P, [%1], %2;\n\t"
+      "{\n\t.reg .pred P;\n\tmbarrier.try_wait.parity.relaxed.cta.shared::cta.b64 P, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, P;\n\t}\n"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -90,19 +90,19 @@ __device__ __forceinline__ bool mbar_test_wait_relaxed(uint64_t *bar, uint32_t p
   return ok != 0;
 }
 
-// mbar_wait for the waits of a thread that issues tcgen05.mma: polls the
-// phase with relaxed test_wait and, once it has completed, establishes the
+// mbar_wait for the waits of a thread that issues tcgen05.mma: waits for the
+// phase with a relaxed try_wait and, once it has completed, establishes the
 // acquire ordering with fence.acq_rel.cta.  Measured on B200, an acquire
 // test_wait / try_wait between small MMAs stalls the issuing thread until its
-// queued MMAs drain (~270 cycles per wait at 4 MMAs per wait), the relaxed
-// poll plus fence costs ~90.  Same bound and status as mbar_wait.
+// queued MMAs drain (~270 cycles per wait at 4 MMAs per wait); the relaxed
+// wait plus fence costs ~90.  Same bound and status as mbar_wait.
 __device__ __forceinline__ bool mbar_wait_relaxed(uint64_t *bar, uint32_t parity, unsigned *status) {
-  if (!mbar_test_wait_relaxed(bar, parity)) {
+  if (!mbar_try_wait_relaxed(bar, parity)) {
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
       bool done = false;
 #pragma unroll 1
-      for (int i = 0; i < 64 && !done; ++i) done = mbar_test_wait_relaxed(bar, parity);
+      for (int i = 0; i < 32 && !done; ++i) done = mbar_try_wait_relaxed(bar, parity);
       if (done) break;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         atomicOr(status, kStatusTimeout);
