@@ -73,9 +73,9 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 PROFILED_TRAFFIC = {
     "attn_prefill.cu": {"sha1": "bb501558ebeb19bc821a219788ea5b8e5481a8d1", "bytes": 604.078848e6 + 185.454080e6,
                         "how": "ncu capture at the timed size (B=1 H=96 T=8192)"},
-    "attn_latent_tc.cu": {"sha1": "c5244ae68f0d84b6ec11dcbad46f5d696cedb52e", "bytes": 640.111616e6 * 8 + 36.986112e6,
-                          "how": "ncu capture at L=16384, reads scaled x8 to L=131072 (cache traffic grows with L), "
-                                 "partial-state writes unscaled"},
+    "attn_latent_tc.cu": {"sha1": "e6998d11df42c2c24cabc5ebff89bf65c7024b85", "bytes": 544.882176e6 * 8 + 32.930048e6,
+                          "how": "ncu capture of latent_decode_kernel at L=16384, reads scaled x8 to L=131072 (cache "
+                                 "traffic grows with L), partial-state writes unscaled"},
 }
 
 
