@@ -42,6 +42,12 @@ METRIC = "prefill attention TFLOP/s & decode latent-cache GB/s, % of B200 roofli
 P_B, P_H, P_T, D = 1, 96, 8192, 128
 DEC_B, DEC_L, DC, DM = 32, 131072, 512, 12288
 L_B, L_T = 2, 4096   # --workload layer: full layer prefill
+# --workload sweep: context lengths of the "Foundations" page's cost table (8K, 128K, 1M);
+# prefill at B=1 with SWEEP_H heads (the per-head cost is what scales), decode at B=SWEEP_B
+SWEEP_T = (8192, 131072, 1048576)
+SWEEP_H = 8
+SWEEP_B = 4
+SWEEP_PAGE = {"dot_products_per_head": (3.2e7, 8.2e9, 5.2e11), "kv_cache": (1, 16, 128)}
 
 
 def prefill_flops(B=P_B, H=P_H, T=P_T):
@@ -417,6 +423,82 @@ def timed(fn_list, steps, world):
     return total, per
 
 
+def run_sweep(args, rank, world, local, peaks):
+    """Long-context sweep: causal prefill attention (B=1, SWEEP_H heads) and latent-cache
+    decode (B=SWEEP_B, 96 heads, d_c=512) at each length of SWEEP_T, each timed with CUDA
+    events after W warm-up calls; K per size is as many calls as fit ~2 s (at most --steps)."""
+    import torch
+
+    import causal_head_latent_b200 as g
+    from synth_inputs import Draw, prefill_qkv
+
+    def time_fn(fn, launches):
+        for _ in range(args.warmup):
+            fn()
+        g.gmla_get_device_status()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        steps = max(1, min(args.steps, int(2000.0 / max(e0.elapsed_time(e1), 1e-3))))
+        total, _ = timed([fn], steps, world)
+        g.gmla_get_device_status()
+        return max_over_ranks(total, world) / steps, steps * launches
+
+    rows, launches = [], 0
+    clk = ClockSampler(local)
+    clk.start()
+    for i, T in enumerate(SWEEP_T):
+        inp = prefill_qkv(900 + i, 1, T, SWEEP_H)
+        Q, K, V = (dev(inp[k]) for k in ("Q", "K", "V"))
+        del inp
+        O = torch.empty_like(Q)
+        p_ms, n = time_fn(lambda: g.gmla_attend_prefill(Q, K, V, O, causal=True), 1)
+        launches += n
+        del Q, K, V, O
+        dr = Draw(950 + i)
+        H, d = DM // D, DM
+        q = dev(dr.normal((SWEEP_B, d)))
+        Wk = dev(dr.normal((d, DC), 1 / np.sqrt(DC)))
+        Wv = dev(dr.normal((d, DC), 1 / np.sqrt(DC)))
+        C = dev(dr.normal((SWEEP_B, T, DC)))
+        Od = torch.empty(SWEEP_B, d, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(g.gmla_attend_decode_workspace_size(SWEEP_B, T, H, DC), dtype=torch.uint8, device="cuda")
+        d_ms, n = time_fn(lambda: g.gmla_attend_decode(q, C, T, Wk, Wv, Od, H, workspace=ws), 3)
+        launches += n
+        del q, Wk, Wv, C, Od, ws
+        torch.cuda.empty_cache()
+        pf = prefill_flops(1, SWEEP_H, T)
+        db = decode_bytes(SWEEP_B, T)
+        rows.append({"T": T, "dot_products_per_head": T * (T + 1) / 2,
+                     "prefill_ms": p_ms, "prefill_tflops": pf / (p_ms / 1e3) / 1e12,
+                     "prefill_frac_of_sustained_bf16": pf / (p_ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                     "decode_ms": d_ms, "decode_gbs": db / (d_ms / 1e3) / 1e9,
+                     "decode_frac_of_hbm": db / (d_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "cache_bytes_per_sequence": T * DC * 2})
+    clocks = clk.stop()
+    ratios = {}
+    for a, b in ((0, 1), (1, 2)):
+        ta, tb = SWEEP_T[a], SWEEP_T[b]
+        lab = lambda t: f"{t // 1048576}M" if t % 1048576 == 0 else f"{t // 1024}K"
+        key = f"{lab(ta)}->{lab(tb)}"
+        ratios[key] = {"dot_products": rows[b]["dot_products_per_head"] / rows[a]["dot_products_per_head"],
+                       "prefill_time": rows[b]["prefill_ms"] / rows[a]["prefill_ms"],
+                       "kv_cache": tb / ta, "decode_time": rows[b]["decode_ms"] / rows[a]["decode_ms"]}
+    line = {"metric": "long-context sweep: causal prefill attention TFLOP/s and latent-cache decode time vs context "
+                      "length (8K, 128K, 1M)",
+            "value": rows[-1]["prefill_tflops"], "unit": "TFLOP/s", "n_gpus": world, "steps": None,
+            "warmup": args.warmup, "ms_per_step": rows[-1]["prefill_ms"] + rows[-1]["decode_ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"causal prefill attention B=1 H={SWEEP_H} D_h={D} and latent-cache decode "
+                                   f"B={SWEEP_B} H=96 d_c={DC} at T = L = 8192, 131072, 1048576",
+                       "l2": "inputs larger than L2 at 128K and 1M; at 8K the decode cache (33.5 MB) fits in L2"},
+            "clocks": clocks, "gpu_launches": launches, "sweep": rows, "ratios": ratios, "pages": SWEEP_PAGE}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     global DEC_L
     ap = argparse.ArgumentParser()
@@ -425,7 +507,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--parts", default="all", choices=["all", "prefill", "decode"])
-    ap.add_argument("--workload", default="step", choices=["step", "layer"])
+    ap.add_argument("--workload", default="step", choices=["step", "layer", "sweep"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--dec-L", type=int, default=DEC_L,
@@ -444,6 +526,10 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     import causal_head_latent_b200 as g
     peaks = load_peaks()
+
+    if args.workload == "sweep":
+        run_sweep(args, rank, world, local, peaks)
+        return
 
     if args.workload == "layer":
         part = LayerPart(4)

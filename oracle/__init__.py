@@ -234,12 +234,14 @@ def decode_latent(q, cache, L, W_k, W_v, num_heads, G=None, scale=None, heads=No
     D = d // H
     Wk = widen(W_k)
     Wv = widen(W_v)
-    Cw = widen(cache)
     out = np.full((B, d), np.nan)
     wts = np.zeros((B, H, L)) if want_weights else None
     pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    wide = {}  # sequences widened to float64 on first use (the cache can be many GB)
     for b, h in pairs:
-        Cb = np.ascontiguousarray(Cw[b, :L])
+        if b not in wide:
+            wide[b] = widen(np.ascontiguousarray(cache[b, :L]))
+        Cb = wide[b]
         Kh = linear(Cb, Wk[h * D:(h + 1) * D])          # [L, D]
         Vh = linear(Cb, Wv[h * D:(h + 1) * D])
         qh = qd[b, h * D:(h + 1) * D].reshape(1, 1, 1, D)
