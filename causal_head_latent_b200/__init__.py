@@ -54,6 +54,11 @@ lib.gmla_attend_decode.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _
 lib.gmla_attend_decode.restype = _st
 lib.gmla_attend_decode_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
 lib.gmla_attend_decode_workspace_size.restype = _sz
+lib.gmla_attend_decode_varlen.argtypes = [_p, _p, _i64, _i64, _p, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p, _p,
+                                          _p, _p, _sz, _p]
+lib.gmla_attend_decode_varlen.restype = _st
+lib.gmla_attend_decode_varlen_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
+lib.gmla_attend_decode_varlen_workspace_size.restype = _sz
 lib.gmla_attend_decode_noalloc.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p,
                                            _p, _p, _p]
 lib.gmla_attend_decode_noalloc.restype = _st
@@ -201,6 +206,30 @@ def gmla_attend_decode(Q, C, L, W_k, W_v, O, num_heads, scale=0.0, G=None, weigh
     code = lib.gmla_attend_decode(_ptr(Q), _ptr(C), B, Lmax, L, H, D, d_c, _ptr(W_k), _ptr(W_v), float(scale),
                                   _ptr(G), _ptr(O), _ptr(weights), wp, wb, _stream(stream))
     return _check(code, "gmla_attend_decode") if check else code
+
+
+def gmla_attend_decode_varlen_workspace_size(B, cache_len_max, H, d_c) -> int:
+    return lib.gmla_attend_decode_varlen_workspace_size(B, cache_len_max, H, d_c)
+
+
+def gmla_attend_decode_varlen(Q, C, lens, W_k, W_v, O, num_heads, scale=0.0, G=None, weights=None, workspace=None,
+                              stream=None, check=True):
+    """Q, O, G [B, H*D]; C [B, cache_len_max, d_c]; lens: B host integers, sequence b
+    sees cache rows 0..lens[b]-1 (see include/gmla.h)."""
+    for n, t in (("Q", Q), ("C", C), ("W_k", W_k), ("W_v", W_v), ("O", O), ("G", G)):
+        _bf16(t, n)
+    B, d = Q.shape
+    H = int(num_heads)
+    D = d // H
+    _, Lmax, d_c = C.shape
+    lens_arr = (ctypes.c_int64 * B)(*[int(x) for x in lens])
+    if len(lens) != B:
+        raise ValueError("lens needs one length per sequence")
+    wp, wb = _ws(workspace)
+    code = lib.gmla_attend_decode_varlen(_ptr(Q), _ptr(C), B, Lmax, ctypes.cast(lens_arr, _p), H, D, d_c, _ptr(W_k),
+                                         _ptr(W_v), float(scale), _ptr(G), _ptr(O), _ptr(weights), wp, wb,
+                                         _stream(stream))
+    return _check(code, "gmla_attend_decode_varlen") if check else code
 
 
 def gmla_attend_decode_noalloc_max_bytes() -> int:

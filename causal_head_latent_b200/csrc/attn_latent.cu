@@ -12,6 +12,7 @@
 //   combine  exact log-sum-exp merge of the splits, c^ = acc / l, then
 //            o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store.
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -20,7 +21,8 @@ namespace gmla {
 
 int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
                      int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l, float *part_acc,
-                     float *weights, unsigned *status, cudaStream_t stream);
+                     float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens, unsigned *status,
+                     cudaStream_t stream);
 int latent_tc_tile_keys();
 
 namespace latent {
@@ -104,7 +106,10 @@ __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
     const float *acc = P.part_acc + ((size_t)(b0 + bb) * P.H + h) * dc + c;
     const size_t split_stride = (size_t)P.B * P.H * dc;
     float a = 0.f;
-    for (int s = 0; s < S; ++s) a = fmaf(wsp[bb * S + s], acc[s * split_stride], a);
+    for (int s = 0; s < S; ++s) {
+      const float ws = wsp[bb * S + s];
+      if (ws != 0.f) a = fmaf(ws, acc[s * split_stride], a);  // an empty split left no acc
+    }
     chat[i] = a;
   }
   __syncthreads();
@@ -149,6 +154,16 @@ __global__ void weights_fix_kernel(float *w, const float *lse2, int BH, int L) {
   const size_t n = (size_t)BH * L;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
     w[i] = fast_exp2(w[i] - lse2[i / L]);
+}
+
+// Per-sequence lengths: rows of [B, H, Lmax]; columns at or past lens[b] are 0.
+__global__ void weights_fix_varlen_kernel(float *w, const float *lse2, const int *lens, int H, int BH, long long Lmax) {
+  const size_t n = (size_t)BH * Lmax;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / Lmax;
+    const long long col = (long long)(i % Lmax);
+    w[i] = col < lens[r / H] ? fast_exp2(w[i] - lse2[r]) : 0.f;
+  }
 }
 
 }  // namespace latent
@@ -196,6 +211,13 @@ size_t latent_workspace_bytes(long long B, long long L, long long H, long long d
   return latent_workspace_bytes_for(B, H, dc, S);
 }
 
+// With per-sequence lengths the plan follows cache_len_max, and the workspace
+// also holds one 128-byte tensor map and one int32 length per sequence.
+size_t latent_varlen_workspace_bytes(long long B, long long cache_len_max, long long H, long long dc) {
+  return latent_workspace_bytes(B, cache_len_max, H, dc) + align256((size_t)B * sizeof(CUtensorMap)) +
+         align256((size_t)B * sizeof(int));
+}
+
 // The three launches for a given split plan (S splits of kps keys) and workspace.
 static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaStream_t stream) {
   using namespace latent;
@@ -209,6 +231,28 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
   float *pacc = reinterpret_cast<float *>(ws);
   ws += align256(sizeof(float) * (size_t)S * a.B * a.H * a.dc);
   float *lse2 = reinterpret_cast<float *>(ws);
+  ws += align256(sizeof(float) * (size_t)a.B * a.H);
+  CUtensorMap *maps = nullptr;
+  int *lens_dev = nullptr;
+  if (a.lens) {
+    // per-sequence 2-D latent maps (d_c, lens[b]) and lengths, copied before the launches
+    maps = reinterpret_cast<CUtensorMap *>(ws);
+    ws += align256((size_t)a.B * sizeof(CUtensorMap));
+    lens_dev = reinterpret_cast<int *>(ws);
+    std::vector<CUtensorMap> hm((size_t)a.B);
+    std::vector<int> hl((size_t)a.B);
+    for (int b = 0; b < a.B; ++b) {
+      const long long dims[2] = {a.dc, a.lens[b]}, strides[1] = {a.dc};
+      const unsigned box[2] = {64, (unsigned)latent_tc_tile_keys()};
+      if (!make_tmap_bf16(&hm[b], a.C + (size_t)b * a.cache_len_max * a.dc, 2, dims, strides, box)) return -1;
+      hl[b] = (int)a.lens[b];
+    }
+    // pageable sources: the copies are staged before cudaMemcpyAsync returns
+    if (cudaMemcpyAsync(maps, hm.data(), hm.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(lens_dev, hl.data(), hl.size() * sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return -1;
+  }
 
   {
     const size_t shm = sizeof(float) * a.B * HD;
@@ -228,7 +272,9 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     const long long dcm[3] = {a.dc, a.L, a.B}, scm[2] = {a.dc, a.cache_len_max * a.dc};
     const unsigned bc[3] = {64, (unsigned)latent_tc_tile_keys(), 1};
     if (!make_tmap_bf16(&tc, a.C, 3, dcm, scm, bc)) return -1;
-    if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, a.status, stream) != 0)
+    const int w_ld = a.lens ? (int)a.cache_len_max : a.L;
+    if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, w_ld, maps,
+                         lens_dev, a.status, stream) != 0)
       return -1;
   }
   {
@@ -246,13 +292,17 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     P.lse2 = lse2;
     combine_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), CT, sizeof(float) * (CB * a.dc + CB * S), stream>>>(P);
   }
-  if (a.weights) weights_fix_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, a.B * a.H, a.L);
+  if (a.weights && a.lens)
+    weights_fix_varlen_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, lens_dev, a.H, a.B * a.H,
+                                                                 a.cache_len_max);
+  else if (a.weights)
+    weights_fix_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, a.B * a.H, a.L);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
   int S, kps;
-  latent_plan(a.B, a.L, &S, &kps);
+  latent_plan(a.B, a.lens ? a.cache_len_max : a.L, &S, &kps);
   return launch_attend_latent_plan(a, S, kps, stream);
 }
 

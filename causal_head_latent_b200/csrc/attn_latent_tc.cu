@@ -96,7 +96,13 @@ struct Params {
   long long Lmax;
   int B, L, H, dc, n_splits, keys_per_split;
   float *part_m, *part_l, *part_acc;  // [S,B,H], [S,B,H], [S,B,H,512]
-  float *weights;                     // optional raw log2-domain scores [B,H,L]
+  float *weights;                     // optional raw log2-domain scores [B,H,w_ld]
+  int w_ld;                           // row stride of weights (L, or Lmax with per-sequence lengths)
+  // Per-sequence lengths (null: every sequence has L rows): lens[b] rows of
+  // sequence b are visible, read through tmC_seq[b], a 2-D map (d_c, lens[b])
+  // whose row extent makes a ragged last tile read zeros past lens[b].
+  const CUtensorMap *tmC_seq;
+  const int *lens;
   unsigned *status;
 };
 
@@ -159,9 +165,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int b = blockIdx.x / p.n_splits;
   const int split = blockIdx.x % p.n_splits;
+  const int Lb = p.lens ? p.lens[b] : p.L;
   const int k_begin = split * p.keys_per_split;
-  const int k_end = min(p.L, k_begin + p.keys_per_split);
-  const int n_tiles = (k_end - k_begin + KT - 1) / KT;  // >= 1 (the host leaves no split empty)
+  const int k_end = min(Lb, k_begin + p.keys_per_split);
+  if (k_end <= k_begin) {
+    // A split past the end of a shorter sequence: an empty partial state,
+    // which the combine skips.  The whole CTA leaves before any barrier.
+    const size_t rec = ((size_t)split * p.B + b) * p.H;
+    for (int h = threadIdx.x; h < p.H; h += NUM_THREADS) {
+      p.part_m[rec + h] = -INFINITY;
+      p.part_l[rec + h] = 0.f;
+    }
+    return;
+  }
+  const int n_tiles = (k_end - k_begin + KT - 1) / KT;  // >= 1
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -188,8 +205,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      const CUtensorMap *mC = p.tmC_seq ? p.tmC_seq + b : &tmC;
+      if (p.tmC_seq) fence_tensormap_acquire(mC);
       tma_prefetch_desc(&tmQt);
-      tma_prefetch_desc(&tmC);
+      tma_prefetch_desc(mC);
       mbar_arrive_expect_tx(bar_q, Q_BYTES);
       for (int kc = 0; kc < NCHUNK; ++kc) tma_load_3d(sq + kc * QCHUNK, &tmQt, bar_q, kc * 64, 0, b);
       // The latents of this split are one contiguous range; a short L2
@@ -212,8 +231,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         uint64_t *fb = q < NEARLY_PAIRS ? &full_e[j % NTB] : &full_l[j % NTB];
         mbar_arrive_expect_tx(fb, 2 * CCHUNK);
-        for (int h2 = 0; h2 < 2; ++h2)
-          tma_load_3d(sc + (2 * ps + h2) * CCHUNK, &tmC, fb, (2 * q + h2) * 64, k_begin + j * KT, b);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (p.tmC_seq)
+            tma_load_2d(sc + (2 * ps + h2) * CCHUNK, mC, fb, (2 * q + h2) * 64, k_begin + j * KT);
+          else
+            tma_load_3d(sc + (2 * ps + h2) * CCHUNK, mC, fb, (2 * q + h2) * 64, k_begin + j * KT, b);
+        }
         issued = g + 1;
       }
       // Error path: let the copies still in flight land before the CTA exits
@@ -290,7 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float m_used = -INFINITY, l = 0.f;
     uint8_t *prow = sp + h * 128;
     const int sw = h & 7;
-    float *wrow = (p.weights && head_ok) ? p.weights + ((size_t)b * p.H + h) * (size_t)p.L : nullptr;
+    float *wrow = (p.weights && head_ok) ? p.weights + ((size_t)b * p.H + h) * (size_t)p.w_ld : nullptr;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int sb = j & 1;
@@ -421,7 +444,8 @@ int latent_tc_tile_keys() { return latent_tc::KT; }
 
 int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
                      int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l, float *part_acc,
-                     float *weights, unsigned *status, cudaStream_t stream) {
+                     float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens, unsigned *status,
+                     cudaStream_t stream) {
   using namespace latent_tc;
   auto kern = latent_decode_kernel;
   const size_t smem = smem_bytes();
@@ -443,6 +467,9 @@ int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint
   p.part_l = part_l;
   p.part_acc = part_acc;
   p.weights = weights;
+  p.w_ld = w_ld;
+  p.tmC_seq = tmC_seq;
+  p.lens = lens;
   p.status = status;
   kern<<<B * n_splits, NUM_THREADS, smem, stream>>>(tmQt, tmC, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

@@ -337,6 +337,40 @@ gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B
   return launch_attend_latent(a, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ decode with per-sequence lengths
+
+size_t gmla_attend_decode_varlen_workspace_size(int64_t B, int64_t cache_len_max, int64_t H, int64_t d_c) {
+  if (B <= 0 || cache_len_max <= 0 || H <= 0 || d_c <= 0) return 0;
+  return latent_varlen_workspace_bytes(B, cache_len_max, H, d_c);
+}
+
+gmla_status gmla_attend_decode_varlen(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B, int64_t cache_len_max,
+                                      const int64_t *lens, int64_t H, int64_t D_h, int64_t d_c, const gmla_bf16 *W_k,
+                                      const gmla_bf16 *W_v, float scale, const gmla_bf16 *G, gmla_bf16 *O,
+                                      float *weights, void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
+  if (!Q || !C || !W_k || !W_v || !O || !lens) return GMLA_ERR_ARG;
+  if (B <= 0 || H <= 0 || D_h <= 0 || d_c <= 0 || cache_len_max < 1) return GMLA_ERR_ARG;
+  for (int64_t b = 0; b < B; ++b)
+    if (lens[b] < 1 || lens[b] > cache_len_max) return GMLA_ERR_ARG;
+  const void *ptrs[] = {Q, C, W_k, W_v, G, O, workspace};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (D_h != 128 || d_c % 64 != 0 || d_c > 512 || H > 96) return GMLA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || cache_len_max > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  const size_t need = latent_varlen_workspace_bytes(B, cache_len_max, H, d_c);
+  if (!workspace || workspace_bytes < need) return GMLA_ERR_WORKSPACE;
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D_h);
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  LatentArgs a{};
+  a.Q = Q; a.C = C; a.Wk = W_k; a.Wv = W_v; a.G = G; a.O = O; a.weights = weights;
+  a.cache_len_max = cache_len_max;
+  a.B = (int)B; a.L = (int)cache_len_max; a.H = (int)H; a.dc = (int)d_c;
+  a.scale = scale; a.workspace = workspace; a.status = st;
+  a.lens = reinterpret_cast<const long long *>(lens);
+  return launch_attend_latent(a, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ decode without a caller workspace
 
 size_t gmla_attend_decode_noalloc_max_bytes(void) { return latent_noalloc_scratch_bytes(); }

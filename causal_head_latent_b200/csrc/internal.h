@@ -71,9 +71,13 @@ struct LatentArgs {
   float scale;
   void *workspace;
   unsigned *status;
+  // Optional per-sequence lengths (host array of B values in 1..cache_len_max);
+  // when set, L is ignored and the split plan and workspace follow cache_len_max.
+  const long long *lens = nullptr;
 };
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream);
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc);
+size_t latent_varlen_workspace_bytes(long long B, long long cache_len_max, long long H, long long dc);
 // Same launches with the scratch in a fixed device array of this library
 // (no workspace argument).  Returns 0, -1 (CUDA error) or -3 (too large).
 int launch_attend_latent_noalloc(const LatentArgs &a, cudaStream_t stream);

@@ -162,6 +162,13 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
+// Make a tensor map that ordinary (generic-proxy) writes placed in global
+// memory -- here a copy from the host before the launch -- visible to the
+// tensor-map proxy that TMA reads it through, rather than a stale cached copy.
+__device__ __forceinline__ void fence_tensormap_acquire(const void *map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+}
+
 // Fetch `bytes` (multiple of 16, 16-byte aligned address) of global memory into L2.
 __device__ __forceinline__ void prefetch_l2_bulk(const void *gptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");

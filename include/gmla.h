@@ -160,6 +160,37 @@ GMLA_API gmla_status gmla_attend_decode(const gmla_bf16 *Q, const gmla_bf16 *C, 
 GMLA_API size_t gmla_attend_decode_workspace_size(int64_t B, int64_t L, int64_t H, int64_t d_c);
 
 /*
+ * gmla_attend_decode_varlen -- gmla_attend_decode over a batch whose sequences
+ * hold different numbers of cached latents: the two-dimensional padding mask
+ * of the "Kimi K2 - Construct causal mask" page (positions past a sequence's
+ * length are padding, combined with the causal mask) in its length form.
+ * Sequence b attends to
+ * rows 0..lens[b]-1 of its cache, its new latent at row lens[b]-1 (the query
+ * position is the cached length: that page's position ids start at the past
+ * length).  Rows at or past lens[b] are never read as data: they may hold
+ * anything, NaN included.
+ *
+ *  lens    HOST array of B lengths, 1 <= lens[b] <= cache_len_max; read
+ *          during the call only.  The other arguments are those of
+ *          gmla_attend_decode.
+ *  weights optional float32 [B, H, cache_len_max]; columns at or past lens[b]
+ *          are written as 0.
+ *  workspace >= gmla_attend_decode_varlen_workspace_size(B, cache_len_max,
+ *          H, d_c) bytes; it also receives one tensor map and one length per
+ *          sequence (copied from the host on `stream` before the launches).
+ * Errors: GMLA_ERR_ARG for a null pointer or a length outside 1..cache_len_max,
+ * the rest as gmla_attend_decode.
+ */
+GMLA_API gmla_status gmla_attend_decode_varlen(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B,
+                                              int64_t cache_len_max, const int64_t *lens, int64_t H,
+                                              int64_t D_h, int64_t d_c, const gmla_bf16 *W_k,
+                                              const gmla_bf16 *W_v, float scale, const gmla_bf16 *G,
+                                              gmla_bf16 *O, float *weights, void *workspace,
+                                              size_t workspace_bytes, gmla_stream_t stream);
+GMLA_API size_t gmla_attend_decode_varlen_workspace_size(int64_t B, int64_t cache_len_max, int64_t H,
+                                                         int64_t d_c);
+
+/*
  * gmla_attend_decode_noalloc -- gmla_attend_decode for callers that cannot
  * allocate device memory.  No page has a counterpart: it is a service of this
  * library, not a step of the method.

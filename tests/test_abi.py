@@ -89,6 +89,17 @@ def test_host_validation_without_gpu(gmla):
     assert L.gmla_attend_decode(fake, fake, 2, 100, 100, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 16,
                                 None) == 5
     assert L.gmla_attend_decode_workspace_size(2, 100, 2, 64) > 16
+    # varlen decode: null lens, a zero length, a length past the cache, a short workspace
+    lens = (ctypes.c_int64 * 2)(5, 7)
+    bad0 = (ctypes.c_int64 * 2)(5, 0)
+    bad1 = (ctypes.c_int64 * 2)(5, 101)
+    LV = L.gmla_attend_decode_varlen
+    assert LV(fake, fake, 2, 100, None, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 1 << 30, None) == 1
+    assert LV(fake, fake, 2, 100, bad0, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 1 << 30, None) == 1
+    assert LV(fake, fake, 2, 100, bad1, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 1 << 30, None) == 1
+    assert LV(fake, fake, 2, 100, lens, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 16, None) == 5
+    assert L.gmla_attend_decode_varlen_workspace_size(2, 100, 2, 64) > L.gmla_attend_decode_workspace_size(2, 100, 2,
+                                                                                                          64)
     # an empty query set is a no-op that launches nothing
     assert L.gmla_attend_prefill(fake, s, fake, s, fake, s, 1, 2, 0, 300, 128, 1, 0.0, None, fake, s, None, None,
                                  None) == 0

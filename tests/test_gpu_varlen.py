@@ -1,0 +1,98 @@
+"""GPU parity of the per-sequence-length decode (gmla_attend_decode_varlen): the
+two-dimensional padding mask of the "Kimi K2 - Construct causal mask" page in
+length form, each sequence checked against the oracle on its own visible rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from synth_inputs import Draw
+from tests.gpu_util import ROW_SUM, assert_parity, bits, f64, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    import causal_head_latent_b200 as gm
+    return gm
+
+
+def _inputs(seed, B, Lmax, H, d_c):
+    d = 128 * H
+    dr = Draw(seed)
+    q = dr.normal((B, d))
+    cache = dr.normal((B, Lmax, d_c))
+    Wk = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Wv = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Gl = dr.normal((B, d))
+    return q, cache, Wk, Wv, Gl
+
+
+def test_decode_varlen_matches_oracle_per_sequence(g):
+    """Lengths 1, a partial tile, one tile, a multi-split length and the full cache;
+    rows past each length hold NaN."""
+    B, Lmax, H, d_c = 5, 4200, 8, 512
+    lens = [1, 47, 48, 1000, 4200]
+    d = 128 * H
+    q, cache, Wk, Wv, Gl = _inputs(1201, B, Lmax, H, d_c)
+    dirty = cache.copy()
+    for b, n in enumerate(lens):
+        dirty[b, n:, :] = 0x7FC0  # bfloat16 quiet NaN past the sequence's length
+    O = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    W = torch.full((B, H, Lmax), float("nan"), device="cuda")
+    work = torch.empty(g.gmla_attend_decode_varlen_workspace_size(B, Lmax, H, d_c), dtype=torch.uint8, device="cuda")
+    g.gmla_attend_decode_varlen(to_dev(q), to_dev(dirty), lens, to_dev(Wk), to_dev(Wv), O, H, G=to_dev(Gl),
+                                weights=W, workspace=work)
+    g.gmla_get_device_status()
+    got, w = f64(O), f64(W)
+    assert np.all(np.isfinite(got))
+    for b, n in enumerate(lens):
+        ref, wref = orc.decode_latent(q[b:b + 1], np.ascontiguousarray(cache[b:b + 1, :n]), n, Wk, Wv, H,
+                                      G=Gl[b:b + 1], want_weights=True)
+        assert_parity(got[b:b + 1], ref, f"varlen decode sequence {b} (length {n})")
+        assert np.abs(w[b, :, :n].sum(-1) - 1.0).max() <= ROW_SUM
+        assert np.all(w[b, :, n:] == 0.0)
+        # relative bound: see test_attend_decode_matches_oracle (bfloat16 absorbed query)
+        assert np.all(np.abs(w[b, :, :n] - wref[0]) <= 2e-5 + 1e-2 * wref[0])
+
+
+def test_decode_varlen_equal_lengths_equals_uniform(g):
+    """All lengths equal to cache_len_max: the same split plan and the same data as
+    gmla_attend_decode, so the outputs match bit for bit."""
+    B, L, H, d_c = 3, 2049, 16, 512
+    d = 128 * H
+    q, cache, Wk, Wv, Gl = _inputs(1202, B, L, H, d_c)
+    t = {k: to_dev(v) for k, v in (("q", q), ("C", cache), ("Wk", Wk), ("Wv", Wv), ("G", Gl))}
+    O1 = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    O2 = torch.empty_like(O1)
+    w1 = torch.empty(g.gmla_attend_decode_workspace_size(B, L, H, d_c), dtype=torch.uint8, device="cuda")
+    w2 = torch.empty(g.gmla_attend_decode_varlen_workspace_size(B, L, H, d_c), dtype=torch.uint8, device="cuda")
+    g.gmla_attend_decode(t["q"], t["C"], L, t["Wk"], t["Wv"], O1, H, G=t["G"], workspace=w1)
+    g.gmla_attend_decode_varlen(t["q"], t["C"], [L] * B, t["Wk"], t["Wv"], O2, H, G=t["G"], workspace=w2)
+    g.gmla_get_device_status()
+    assert np.array_equal(bits(O1), bits(O2))
+
+
+def test_decode_varlen_full_size_sampled(g):
+    """B=32 sequences of mixed lengths up to 131072 cached latents, 96 heads, d_c=512,
+    checked on sampled (b, h) pairs."""
+    B, Lmax, H, d_c = 32, 131072, 96, 512
+    d = 128 * H
+    rng = np.random.default_rng(1203)
+    lens = [int(x) for x in rng.integers(1, Lmax + 1, B)]
+    lens[3], lens[17] = 1, Lmax
+    q, cache, Wk, Wv, Gl = _inputs(1203, B, Lmax, H, d_c)
+    O = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    work = torch.empty(g.gmla_attend_decode_varlen_workspace_size(B, Lmax, H, d_c), dtype=torch.uint8, device="cuda")
+    g.gmla_attend_decode_varlen(to_dev(q), to_dev(cache), lens, to_dev(Wk), to_dev(Wv), O, H, G=to_dev(Gl),
+                                workspace=work)
+    g.gmla_get_device_status()
+    got = f64(O)
+    assert np.all(np.isfinite(got))
+    for b, h in [(3, 0), (17, 95), (8, 40)]:
+        n = lens[b]
+        ref = orc.decode_latent(q[b:b + 1], np.ascontiguousarray(cache[b:b + 1, :n]), n, Wk, Wv, H, G=Gl[b:b + 1],
+                                heads=[(0, h)])
+        sl = slice(h * 128, (h + 1) * 128)
+        assert_parity(got[b, sl], ref[0, sl], f"varlen full-size b={b} h={h} length {n}")
