@@ -79,7 +79,7 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 PROFILED_TRAFFIC = {
     "attn_prefill.cu": {"sha1": "bb501558ebeb19bc821a219788ea5b8e5481a8d1", "bytes": 604.078848e6 + 185.454080e6,
                         "how": "ncu capture at the timed size (B=1 H=96 T=8192)"},
-    "attn_latent_tc.cu": {"sha1": "e6998d11df42c2c24cabc5ebff89bf65c7024b85", "bytes": 544.882176e6 * 8 + 32.930048e6,
+    "attn_latent_tc.cu": {"sha1": "364762a2d84494c68f2ebb53fa6143c2fc15edc0", "bytes": 544.323328e6 * 8 + 32.472832e6,
                           "how": "ncu capture of latent_decode_kernel at L=16384, reads scaled x8 to L=131072 (cache "
                                  "traffic grows with L), partial-state writes unscaled"},
 }

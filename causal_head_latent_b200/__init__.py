@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "GmlaError", "lib", "library_path",
     "gmla_latent_project", "gmla_latent_project_workspace_size",
-    "gmla_attend_prefill", "gmla_attend_decode", "gmla_attend_decode_workspace_size",
+    "gmla_expand_kv", "gmla_attend_prefill", "gmla_attend_decode", "gmla_attend_decode_workspace_size",
     "gmla_gate_out", "gmla_gate_out_workspace_size", "gmla_get_device_status", "gmla_status_string",
     "gmla_version", "STATUS",
 ]
@@ -46,6 +46,8 @@ lib.gmla_latent_project.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _i64, _p, 
 lib.gmla_latent_project.restype = _st
 lib.gmla_latent_project_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
 lib.gmla_latent_project_workspace_size.restype = _sz
+lib.gmla_expand_kv.argtypes = [_p, _i64, _i64, _i64, _i64, _i64, _p, _p, _i64, _p, _p, _p]
+lib.gmla_expand_kv.restype = _st
 lib.gmla_attend_prefill.argtypes = [_p, _i64x3, _p, _i64x3, _p, _i64x3, _i64, _i64, _i64, _i64, _i64,
                                     ctypes.c_int, ctypes.c_float, _p, _p, _i64x3, _p, _p, _p]
 lib.gmla_attend_prefill.restype = _st
@@ -157,6 +159,17 @@ def gmla_latent_project(X, W_q, W_g, W_c, W_k, W_v, Q=None, G=None, C=None, cach
                                    _ptr(Q), _ptr(G), _ptr(C), cache_len_max, cache_pos, _ptr(K), _ptr(V), wp, wb,
                                    _stream(stream))
     return _check(code, "gmla_latent_project") if check else code
+
+
+def gmla_expand_kv(C, row0, rows, W_k=None, W_v=None, K=None, V=None, stream=None, check=True):
+    """K, V [B, rows, d_model] = C[:, row0:row0+rows] [W_k; W_v]^T; C [B, cache_len_max, d_c]."""
+    for n, t in (("C", C), ("W_k", W_k), ("W_v", W_v), ("K", K), ("V", V)):
+        _bf16(t, n)
+    B, Lmax, d_c = C.shape
+    d_model = (W_k if W_k is not None else W_v).shape[0]
+    code = lib.gmla_expand_kv(_ptr(C), B, Lmax, int(row0), int(rows), d_c, _ptr(W_k), _ptr(W_v), d_model, _ptr(K),
+                              _ptr(V), _stream(stream))
+    return _check(code, "gmla_expand_kv") if check else code
 
 
 def _bthd_strides(t, layout):

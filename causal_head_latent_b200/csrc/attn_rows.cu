@@ -58,7 +58,10 @@ __global__ void __launch_bounds__(THREADS) attn_rows_kernel(const Params P) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
-  for (int s0 = hw; s0 <= lim; s0 += HALF_WARPS * UNROLL) {
+  // The trip count depends only on lim, never on hw: both half-warps of a warp
+  // run every iteration, since the full-warp shuffles below need all 32 lanes.
+  for (int base = 0; base <= lim; base += HALF_WARPS * UNROLL) {
+    const int s0 = base + hw;
     float kf[UNROLL][8], vf[UNROLL][8];
     bool valid[UNROLL];
 #pragma unroll

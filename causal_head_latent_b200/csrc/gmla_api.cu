@@ -248,6 +248,53 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
   return GMLA_OK;
 }
 
+// ------------------------------------------------------------------ K/V expansion of cached latents
+
+gmla_status gmla_expand_kv(const gmla_bf16 *C, int64_t B, int64_t cache_len_max, int64_t row0, int64_t rows,
+                           int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v, int64_t d_model, gmla_bf16 *K,
+                           gmla_bf16 *V, gmla_stream_t stream) {
+  if (!C || (!K && !V) || (K && !W_k) || (V && !W_v)) return GMLA_ERR_ARG;
+  if (B <= 0 || rows <= 0 || row0 < 0 || d_c <= 0 || d_model <= 0 || cache_len_max <= 0 ||
+      row0 + rows > cache_len_max)
+    return GMLA_ERR_ARG;
+  const void *ptrs[] = {C, W_k, W_v, K, V};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (d_model % 128 != 0 || d_c % 64 != 0) return GMLA_ERR_UNSUPPORTED;
+  if (B * rows > 0x7fffffffLL || cache_len_max > 0x7fffffffLL || B > 65535) return GMLA_ERR_UNSUPPORTED;
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  GemmArgs ga{};
+  CUtensorMap tmA, tmB[3];
+  const long long dA[3] = {d_c, row0 + rows, B}, sA[2] = {d_c, cache_len_max * d_c};
+  const unsigned bA[3] = {64, 128, 1};
+  if (!make_tmap_bf16(&tmA, C, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+  ga.a_rows = (int)rows;
+  ga.a_batches = (int)B;
+  ga.a_row0 = (int)row0;
+  ga.K = (int)d_c;
+  ga.status = st;
+  int np = 0;
+  const gmla_bf16 *Ws[2] = {W_k, W_v};
+  gmla_bf16 *Os[2] = {K, V};
+  for (int i = 0; i < 2; ++i) {
+    if (!Os[i]) continue;
+    const long long dB[2] = {d_c, d_model}, sB[1] = {d_c};
+    const unsigned bB[2] = {64, 256};
+    if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+    GemmOut &o = ga.prob[np];
+    o.out = Os[i];
+    o.N = (int)d_model;
+    o.rows_per_b = B * rows;
+    o.sb = 0;
+    o.st = d_model;
+    o.off = 0;
+    ++np;
+  }
+  ga.n_problems = np;
+  return launch_gemm(tmA, tmB, ga, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ attention over explicit Q, K, V
 
 gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_strides[3], const gmla_bf16 *K,

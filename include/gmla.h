@@ -102,6 +102,28 @@ GMLA_API gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t 
 GMLA_API size_t gmla_latent_project_workspace_size(int64_t B, int64_t T, int64_t d_model, int64_t d_c);
 
 /*
+ * gmla_expand_kv -- K = C W_k^T and V = C W_v^T for cached latent rows
+ * [row0, row0 + rows) of every sequence ("Gated MLA" page, "Start from
+ * familiar attention"; implementation-order step 2).  A prefill chunk that
+ * continues a sequence already in the cache attends to all earlier rows too
+ * (its queries sit at positions cache_pos + t, "Kimi K2 - Construct causal
+ * mask" page), and the cache holds only latents, so those rows are expanded
+ * again: gmla_latent_project(X_chunk, cache_pos = P) appends the chunk, then
+ * gmla_expand_kv(row0 = 0, rows = P + T) gives the keys and values that
+ * gmla_attend_prefill(Tq = T, Tk = P + T) needs.
+ *
+ *  C       latent cache [B, cache_len_max, d_c] (input)
+ *  W_k, W_v [d_model, d_c]; either output may be NULL (then its weight too)
+ *  K, V    [B, rows, d_model] outputs
+ * Returns GMLA_ERR_ARG for null required pointers, row0 < 0, rows < 1,
+ * row0 + rows > cache_len_max or misalignment; GMLA_ERR_UNSUPPORTED when
+ * d_model is not a multiple of 128 or d_c not a multiple of 64.
+ */
+GMLA_API gmla_status gmla_expand_kv(const gmla_bf16 *C, int64_t B, int64_t cache_len_max, int64_t row0,
+                                   int64_t rows, int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v,
+                                   int64_t d_model, gmla_bf16 *K, gmla_bf16 *V, gmla_stream_t stream);
+
+/*
  * gmla_attend_prefill -- per-head scaled dot-product attention over explicit
  * Q, K, V, with the causal mask and float32 softmax over keys, optionally
  * followed by the channel gate.  "Gated MLA" page, "Start from familiar

@@ -100,6 +100,10 @@ def test_host_validation_without_gpu(gmla):
     assert LV(fake, fake, 2, 100, lens, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 16, None) == 5
     assert L.gmla_attend_decode_varlen_workspace_size(2, 100, 2, 64) > L.gmla_attend_decode_workspace_size(2, 100, 2,
                                                                                                           64)
+    # expand_kv: range past the cache, no output, d_model not a multiple of 128
+    assert L.gmla_expand_kv(fake, 2, 100, 50, 51, 64, fake, fake, 256, fake, fake, None) == 1
+    assert L.gmla_expand_kv(fake, 2, 100, 0, 10, 64, fake, fake, 256, None, None, None) == 1
+    assert L.gmla_expand_kv(fake, 2, 100, 0, 10, 64, fake, fake, 200, fake, fake, None) == 2
     # an empty query set is a no-op that launches nothing
     assert L.gmla_attend_prefill(fake, s, fake, s, fake, s, 1, 2, 0, 300, 128, 1, 0.0, None, fake, s, None, None,
                                  None) == 0

@@ -106,6 +106,24 @@ def test_decode_softmax_page_shape_full(g):
     assert np.abs(w - wref).max() < 1e-5
 
 
+@pytest.mark.parametrize("Tq,Tk", [(1, 1), (1, 2), (1, 5), (2, 16), (1, 17), (1, 129), (1, 131), (4, 193), (3, 200),
+                                   (1, 1015)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_few_query_rows_matches_oracle(g, Tq, Tk, causal):
+    """Tq <= 4 runs on the CUDA-core rows kernel.  The key counts cover tiny inputs
+    and last-visible-key positions whose residue mod 64 falls on every half-warp
+    pairing (the loop must keep both half-warps of a warp together)."""
+    inp = prefill_qkv(61 + Tk + Tq, 2, Tq, 3, Tk=Tk, gate=True)
+    O, L, W = run_prefill(g, inp, causal=causal, gate=True, lse=True, weights=True)
+    ref, wref, lref = orc.attention(inp["Q"], inp["K"], inp["V"], causal=causal, want_weights=True, want_lse=True)
+    assert_parity(f64(O), orc.gate(ref.reshape(2, Tq, -1), inp["G"]).reshape(ref.shape), "few-query rows")
+    np.testing.assert_allclose(f64(L), lref, atol=5e-4)
+    w = f64(W)
+    assert np.abs(w.sum(-1) - 1.0).max() <= ROW_SUM
+    assert np.all(w[wref == 0.0] == 0.0)
+    assert np.abs(w - wref).max() < 1e-4
+
+
 def test_prefill_8k_full_size_sampled(g):
     """Causal prefill B=1, H=96, T=8192 (the timed launch), checked on sampled rows."""
     T, H = 8192, 96

@@ -87,6 +87,66 @@ def test_layer_chained_matches_oracle(g):
     assert Y.shape == t["X"].shape and Y.dtype == t["X"].dtype
 
 
+@pytest.mark.parametrize("T1,T2", [(300, 200), (128, 1), (1, 257)])
+def test_chunked_prefill_matches_full_layer(g, T1, T2):
+    """Two prefill chunks of the same sequences through the latent cache: the
+    second chunk appends its latents at cache_pos = T1, re-expands K and V for
+    rows 0..T1+T2-1 (gmla_expand_kv) and attends with Tq = T2 < Tk = T1 + T2.
+    Its layer output equals rows T1.. of the oracle's full-sequence layer; the
+    cache and the expanded K, V equal a single-pass run bit for bit."""
+    B, H, d_c = 2, 2, 128
+    T = T1 + T2
+    d = 128 * H
+    w, t = make_layer(29, B, T, d, d_c)
+    C = torch.zeros(B, T, d_c, dtype=torch.bfloat16, device="cuda")
+    Y2 = None
+    for P, Tc in ((0, T1), (T1, T2)):
+        Xc = t["X"][:, P:P + Tc].contiguous()
+        Q = torch.empty(B, Tc, d, dtype=torch.bfloat16, device="cuda")
+        G, O, Y = (torch.empty_like(Q) for _ in range(3))
+        g.gmla_latent_project(Xc, t["W_q"], t["W_g"], t["W_c"], None, None, Q=Q, G=G, C=C, cache_pos=P)
+        K = torch.empty(B, P + Tc, d, dtype=torch.bfloat16, device="cuda")
+        V = torch.empty_like(K)
+        g.gmla_expand_kv(C, 0, P + Tc, W_k=t["W_k"], W_v=t["W_v"], K=K, V=V)
+        g.gmla_attend_prefill(Q.view(B, Tc, H, 128), K.view(B, P + Tc, H, 128), V.view(B, P + Tc, H, 128),
+                              O.view(B, Tc, H, 128), G=G)
+        g.gmla_gate_out(O, t["W_o"], Y)
+        Y2 = Y
+    g.gmla_get_device_status()
+    ref = orc.gated_mla(w["X"], w["W_q"], w["W_c"], w["W_k"], w["W_v"], w["W_g"], w["W_o"], H,
+                        round_boundaries=True)
+    assert_parity(f64(Y2), ref["output"][:, T1:], "second chunk vs full-sequence layer")
+    # single pass: same latents, and expansion of all rows equals the chunked run's last expansion
+    C1 = torch.empty_like(C)
+    K1 = torch.empty(B, T, d, dtype=torch.bfloat16, device="cuda")
+    V1 = torch.empty_like(K1)
+    g.gmla_latent_project(t["X"], None, None, t["W_c"], t["W_k"], t["W_v"], C=C1, K=K1, V=V1)
+    g.gmla_get_device_status()
+    assert np.array_equal(bits(C), bits(C1))
+    assert np.array_equal(bits(K), bits(K1)) and np.array_equal(bits(V), bits(V1))
+
+
+def test_expand_kv_row_range(g):
+    """gmla_expand_kv over an interior row range of a longer cache equals those rows
+    of the full expansion."""
+    B, Lmax, H, d_c = 3, 700, 2, 192
+    d = 128 * H
+    dr = Draw(31)
+    cache = dr.normal((B, Lmax, d_c))
+    Wk = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Wv = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Cd, Wkd, Wvd = to_dev(cache), to_dev(Wk), to_dev(Wv)
+    row0, rows = 133, 400
+    K = torch.empty(B, rows, d, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    g.gmla_expand_kv(Cd, row0, rows, W_k=Wkd, W_v=Wvd, K=K, V=V)
+    g.gmla_get_device_status()
+    ref_k = orc.linear(cache[:, row0:row0 + rows], Wk)
+    ref_v = orc.linear(cache[:, row0:row0 + rows], Wv)
+    assert_parity(f64(K), ref_k, "expanded K")
+    assert_parity(f64(V), ref_v, "expanded V")
+
+
 @pytest.mark.parametrize("B,L,Lmax,H,d_c", [(3, 700, 700, 4, 128), (2, 1, 5, 2, 64), (1, 2049, 3000, 3, 512),
                                              (2, 4163, 4200, 96, 512), (1, 63, 64, 1, 512)])
 def test_attend_decode_matches_oracle(g, B, L, Lmax, H, d_c):
