@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "GmlaError", "lib", "library_path",
     "gmla_latent_project", "gmla_latent_project_workspace_size",
-    "gmla_expand_kv", "gmla_attend_prefill", "gmla_attend_decode", "gmla_attend_decode_workspace_size",
+    "gmla_expand_kv", "gmla_attend_prefill", "gmla_attend_prefill_varlen", "gmla_attend_prefill_varlen_workspace_size",
+    "gmla_attend_decode", "gmla_attend_decode_workspace_size",
     "gmla_gate_out", "gmla_gate_out_workspace_size", "gmla_get_device_status", "gmla_status_string",
     "gmla_version", "STATUS",
 ]
@@ -51,6 +52,11 @@ lib.gmla_expand_kv.restype = _st
 lib.gmla_attend_prefill.argtypes = [_p, _i64x3, _p, _i64x3, _p, _i64x3, _i64, _i64, _i64, _i64, _i64,
                                     ctypes.c_int, ctypes.c_float, _p, _p, _i64x3, _p, _p, _p]
 lib.gmla_attend_prefill.restype = _st
+lib.gmla_attend_prefill_varlen.argtypes = [_p, _i64x3, _p, _i64x3, _p, _i64x3, _i64, _i64, _i64, _i64, _i64, _p, _p,
+                                           ctypes.c_int, ctypes.c_float, _p, _p, _i64x3, _p, _p, _sz, _p]
+lib.gmla_attend_prefill_varlen.restype = _st
+lib.gmla_attend_prefill_varlen_workspace_size.argtypes = [_i64]
+lib.gmla_attend_prefill_varlen_workspace_size.restype = _sz
 lib.gmla_attend_decode.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p, _p, _p,
                                    _p, _sz, _p]
 lib.gmla_attend_decode.restype = _st
@@ -200,6 +206,36 @@ def gmla_attend_prefill(Q, K, V, O, causal=True, scale=0.0, G=None, lse=None, we
                                    _ptr(G), _ptr(O), _bthd_strides(O, layout), _ptr(lse), _ptr(weights),
                                    _stream(stream))
     return _check(code, "gmla_attend_prefill") if check else code
+
+
+def gmla_attend_prefill_varlen_workspace_size(B) -> int:
+    return lib.gmla_attend_prefill_varlen_workspace_size(B)
+
+
+def gmla_attend_prefill_varlen(Q, K, V, O, q_lens, kv_lens, causal=True, scale=0.0, G=None, lse=None, workspace=None,
+                               layout="bthd", stream=None, check=True):
+    """Padded batch: Q, O [B,Tq_max,H,D] (or [B,H,Tq_max,D] with layout='bhtd'); K, V [B,Tk_max,H,D];
+    q_lens, kv_lens: B host integers each (see include/gmla.h)."""
+    for n, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("G", G)):
+        _bf16(t, n)
+    if layout == "bthd":
+        B, Tq, H, D = Q.shape
+        Tk = K.shape[1]
+    else:
+        B, H, Tq, D = Q.shape
+        Tk = K.shape[2]
+    if len(q_lens) != B or len(kv_lens) != B:
+        raise ValueError("q_lens and kv_lens need one length per sequence")
+    if lse is not None and lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
+    ql = (ctypes.c_int64 * B)(*[int(x) for x in q_lens])
+    kl = (ctypes.c_int64 * B)(*[int(x) for x in kv_lens])
+    wp, wb = _ws(workspace)
+    code = lib.gmla_attend_prefill_varlen(_ptr(Q), _bthd_strides(Q, layout), _ptr(K), _bthd_strides(K, layout),
+                                          _ptr(V), _bthd_strides(V, layout), B, H, Tq, Tk, D, ctypes.cast(ql, _p),
+                                          ctypes.cast(kl, _p), int(bool(causal)), float(scale), _ptr(G), _ptr(O),
+                                          _bthd_strides(O, layout), _ptr(lse), wp, wb, _stream(stream))
+    return _check(code, "gmla_attend_prefill_varlen") if check else code
 
 
 def gmla_attend_decode_workspace_size(B, L, H, d_c) -> int:

@@ -59,7 +59,13 @@ struct Params {
   long long o_sb, o_st, o_sh;
   float *lse;
   float *weights;
-  int B, H, Tq, Tk, causal;
+  int B, H, Tq, Tk, causal;  // Tq, Tk: the row strides of G, lse and weights (the maxima with lengths)
+  // Per-sequence lengths (null: every sequence has Tq queries and Tk keys):
+  // sequence b has q_lens[b] query rows and kv_lens[b] keys, read through
+  // maps[3b .. 3b+2], 3-D maps (D, length, H) of Q, K and V whose row extent is
+  // the sequence's length, so rows past it read as zeros.
+  const int *q_lens, *kv_lens;
+  const CUtensorMap *maps;
   int n_ct;          // CTAs (256-row query pairs) per (b, h)
   float scale_log2;  // scale * log2(e)
   unsigned *status;
@@ -88,11 +94,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Number of key tiles query tile `qt` needs (0 when the tile has no valid row).
-__device__ __forceinline__ int kv_tiles(const Params &p, int qt) {
+__device__ __forceinline__ int kv_tiles(int Tq, int Tk, int causal, int qt) {
   const int q0 = qt * BM;
-  if (q0 >= p.Tq) return 0;
-  const int last_row = min(q0 + BM - 1, p.Tq - 1);
-  const int last_key = p.causal ? min(p.Tk - 1, p.Tk - p.Tq + last_row) : (p.Tk - 1);
+  if (q0 >= Tq) return 0;
+  const int last_row = min(q0 + BM - 1, Tq - 1);
+  const int last_key = causal ? min(Tk - 1, Tk - Tq + last_row) : (Tk - 1);
   return last_key / BN + 1;
 }
 
@@ -109,9 +115,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int bh = blockIdx.x / p.n_ct;
   const int ct = p.causal ? (p.n_ct - 1 - blockIdx.x % p.n_ct) : (blockIdx.x % p.n_ct);
   const int b = bh / p.H, h = bh % p.H;
-  const int nkv0 = kv_tiles(p, 2 * ct);
-  const int nkv1 = kv_tiles(p, 2 * ct + 1);
+  const int Tq = p.q_lens ? p.q_lens[b] : p.Tq;  // this sequence's query rows and keys
+  const int Tk = p.kv_lens ? p.kv_lens[b] : p.Tk;
+  const int nkv0 = kv_tiles(Tq, Tk, p.causal, 2 * ct);
+  const int nkv1 = kv_tiles(Tq, Tk, p.causal, 2 * ct + 1);
   const int nkv = max(nkv0, nkv1);
+  // Query pairs past a shorter sequence's rows (per-sequence lengths only):
+  // nothing to compute or store; the whole CTA leaves before any barrier.
+  if (nkv == 0) return;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
@@ -140,26 +151,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      const CUtensorMap *mq = p.maps ? p.maps + 3 * b : &tmQ;
+      const CUtensorMap *mk = p.maps ? p.maps + 3 * b + 1 : &tmK;
+      const CUtensorMap *mv = p.maps ? p.maps + 3 * b + 2 : &tmV;
+      if (p.maps) {
+        fence_tensormap_acquire(mq);
+        fence_tensormap_acquire(mk);
+        fence_tensormap_acquire(mv);
+      }
+      // one 64-column half of a 128-row tile (rows `row`.., head h of sequence b)
+      auto load = [&](void *dst, const CUtensorMap *m, uint64_t *bar, int col, int row) {
+        if (p.maps)
+          tma_load_3d(dst, m, bar, col, row, h);
+        else
+          tma_load_4d(dst, m, bar, col, row, h, b);
+      };
+      tma_prefetch_desc(mq);
+      tma_prefetch_desc(mk);
+      tma_prefetch_desc(mv);
       const int q0 = 2 * ct * BM;
       mbar_arrive_expect_tx(&sm.bar_q, 2 * TILE_BYTES);
       for (int i = 0; i < 2; ++i) {
-        tma_load_4d(sm.q[i], &tmQ, &sm.bar_q, 0, q0 + i * BM, h, b);
-        tma_load_4d(sm.q[i] + CHUNK_BYTES, &tmQ, &sm.bar_q, 64, q0 + i * BM, h, b);
+        load(sm.q[i], mq, &sm.bar_q, 0, q0 + i * BM);
+        load(sm.q[i] + CHUNK_BYTES, mq, &sm.bar_q, 64, q0 + i * BM);
       }
       for (int j = 0; j < nkv; ++j) {
         const int s = j % STAGES, ph = ((j / STAGES) & 1) ^ 1;
         const int k0 = j * BN;
         if (!mbar_wait(&sm.k_empty[s], ph, p.status)) break;
         mbar_arrive_expect_tx(&sm.k_full[s], TILE_BYTES);
-        tma_load_4d(sm.k[s], &tmK, &sm.k_full[s], 0, k0, h, b);
-        tma_load_4d(sm.k[s] + CHUNK_BYTES, &tmK, &sm.k_full[s], 64, k0, h, b);
+        load(sm.k[s], mk, &sm.k_full[s], 0, k0);
+        load(sm.k[s] + CHUNK_BYTES, mk, &sm.k_full[s], 64, k0);
         if (!mbar_wait(&sm.v_empty[s], ph, p.status)) break;
         mbar_arrive_expect_tx(&sm.v_full[s], TILE_BYTES);
-        tma_load_4d(sm.v[s], &tmV, &sm.v_full[s], 0, k0, h, b);
-        tma_load_4d(sm.v[s] + CHUNK_BYTES, &tmV, &sm.v_full[s], 64, k0, h, b);
+        load(sm.v[s], mv, &sm.v_full[s], 0, k0);
+        load(sm.v[s] + CHUNK_BYTES, mv, &sm.v_full[s], 64, k0);
       }
     }
   } else if (warp == 1) {
@@ -225,10 +251,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int n_tiles = wg ? nkv1 : nkv0;
     const int q0 = (2 * ct + wg) * BM;
     const int t = q0 + row;
-    const bool row_valid = t < p.Tq;
-    const int shift = p.Tk - p.Tq;
+    const bool row_valid = t < Tq;
+    const int shift = Tk - Tq;
     const int pos = shift + t;
-    const int lim = p.causal ? min(pos, p.Tk - 1) : (p.Tk - 1);  // last visible key of this row
+    const int lim = p.causal ? min(pos, Tk - 1) : (Tk - 1);  // last visible key of this row
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     float *wrow = (p.weights && row_valid) ? p.weights + (((size_t)b * p.H + h) * p.Tq + t) * (size_t)p.Tk : nullptr;
@@ -246,7 +272,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[c * 32 + i] = tmp[i];
       }
-      const bool need_mask = (k0 + BN > p.Tk) || (p.causal && (k0 + BN - 1 > shift + q0));
+      const bool need_mask = k0 + BN - 1 > lim;  // a key of this tile lies past this row's last visible key
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
@@ -379,6 +405,9 @@ int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CU
   p.H = a.H;
   p.Tq = a.Tq;
   p.Tk = a.Tk;
+  p.q_lens = a.q_lens;
+  p.kv_lens = a.kv_lens;
+  p.maps = a.maps;
   p.causal = a.causal;
   p.n_ct = (a.Tq + 2 * BM - 1) / (2 * BM);
   p.scale_log2 = a.scale * kLog2e;

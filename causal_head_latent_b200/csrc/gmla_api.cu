@@ -9,6 +9,8 @@
 #include <mutex>
 
 #include "../../include/gmla.h"
+#include <vector>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -350,6 +352,82 @@ gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_strides[3], 
   a.lse = lse; a.weights = weights;
   a.B = (int)B; a.H = (int)H; a.Tq = (int)Tq; a.Tk = (int)Tk; a.causal = causal;
   a.scale = scale; a.status = st;
+  return launch_attn_prefill(tq, tk, tv, a, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ attention with per-sequence lengths
+
+size_t gmla_attend_prefill_varlen_workspace_size(int64_t B) {
+  if (B <= 0) return 0;
+  return 3 * (size_t)B * sizeof(CUtensorMap) + 2 * (size_t)B * sizeof(int) + 256;
+}
+
+gmla_status gmla_attend_prefill_varlen(const gmla_bf16 *Q, const int64_t q_strides[3], const gmla_bf16 *K,
+                                       const int64_t k_strides[3], const gmla_bf16 *V, const int64_t v_strides[3],
+                                       int64_t B, int64_t H, int64_t Tq_max, int64_t Tk_max, int64_t D_h,
+                                       const int64_t *q_lens, const int64_t *kv_lens, int causal, float scale,
+                                       const gmla_bf16 *G, gmla_bf16 *O, const int64_t o_strides[3], float *lse,
+                                       void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
+  if (!Q || !K || !V || !O || !q_strides || !k_strides || !v_strides || !o_strides || !q_lens || !kv_lens)
+    return GMLA_ERR_ARG;
+  if (B <= 0 || H <= 0 || Tq_max <= 0 || Tk_max <= 0 || D_h <= 0) return GMLA_ERR_ARG;
+  if (causal != 0 && causal != 1) return GMLA_ERR_ARG;
+  for (int64_t b = 0; b < B; ++b)
+    if (q_lens[b] < 0 || q_lens[b] > Tq_max || kv_lens[b] < 1 || kv_lens[b] > Tk_max || q_lens[b] > kv_lens[b])
+      return GMLA_ERR_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (G && !aligned16(G))) return GMLA_ERR_ARG;
+  for (int i = 0; i < 3; ++i) {
+    if (q_strides[i] <= 0 || k_strides[i] <= 0 || v_strides[i] <= 0 || o_strides[i] <= 0) return GMLA_ERR_ARG;
+    if (q_strides[i] % 8 || k_strides[i] % 8 || v_strides[i] % 8 || o_strides[i] % 8) return GMLA_ERR_ARG;
+  }
+  if (D_h != 128) return GMLA_ERR_UNSUPPORTED;
+  if (B > 0xffff || H > 0xffff || Tk_max > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < gmla_attend_prefill_varlen_workspace_size(B)) return GMLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GMLA_ERR_ARG;
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D_h);
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // per-sequence 3-D maps (D, length, H) and lengths, copied into the workspace
+  uint8_t *ws = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(workspace) + 127) & ~uintptr_t(127));
+  CUtensorMap *maps = reinterpret_cast<CUtensorMap *>(ws);
+  int *lens = reinterpret_cast<int *>(ws + 3 * (size_t)B * sizeof(CUtensorMap));
+  std::vector<CUtensorMap> hm(3 * (size_t)B);
+  std::vector<int> hl(2 * (size_t)B);
+  const unsigned box[3] = {64, 128, 1};
+  for (int64_t b = 0; b < B; ++b) {
+    const gmla_bf16 *base[3] = {Q + b * q_strides[0], K + b * k_strides[0], V + b * v_strides[0]};
+    const int64_t *str[3] = {q_strides, k_strides, v_strides};
+    const long long len[3] = {q_lens[b] > 0 ? q_lens[b] : 1, kv_lens[b], kv_lens[b]};
+    for (int i = 0; i < 3; ++i) {
+      const long long d[3] = {128, len[i], H}, sd[2] = {str[i][1], str[i][2]};
+      if (!make_tmap_bf16(&hm[3 * b + i], base[i], 3, d, sd, box)) return GMLA_ERR_CUDA;
+    }
+    hl[b] = (int)q_lens[b];
+    hl[B + b] = (int)kv_lens[b];
+  }
+  // pageable sources: the copies are staged before cudaMemcpyAsync returns
+  if (cudaMemcpyAsync(maps, hm.data(), hm.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(lens, hl.data(), hl.size() * sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return GMLA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;  // unused by the kernel when maps are given; encoded for a valid parameter block
+  const unsigned box4[4] = {64, 128, 1, 1};
+  {
+    const long long d[4] = {128, Tq_max, H, B}, sd[3] = {q_strides[1], q_strides[2], q_strides[0]};
+    if (!make_tmap_bf16(&tq, Q, 4, d, sd, box4)) return GMLA_ERR_CUDA;
+    const long long dk[4] = {128, Tk_max, H, B}, sk[3] = {k_strides[1], k_strides[2], k_strides[0]};
+    if (!make_tmap_bf16(&tk, K, 4, dk, sk, box4)) return GMLA_ERR_CUDA;
+    const long long sv[3] = {v_strides[1], v_strides[2], v_strides[0]};
+    if (!make_tmap_bf16(&tv, V, 4, dk, sv, box4)) return GMLA_ERR_CUDA;
+  }
+  PrefillArgs a{};
+  a.G = G; a.O = O;
+  for (int i = 0; i < 3; ++i) a.o_strides[i] = o_strides[i];
+  a.lse = lse; a.weights = nullptr;
+  a.B = (int)B; a.H = (int)H; a.Tq = (int)Tq_max; a.Tk = (int)Tk_max; a.causal = causal;
+  a.scale = scale; a.status = st;
+  a.q_lens = lens; a.kv_lens = lens + B; a.maps = maps;
   return launch_attn_prefill(tq, tk, tv, a, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
 }
 

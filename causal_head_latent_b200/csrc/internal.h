@@ -22,6 +22,10 @@ struct PrefillArgs {
   int B, H, Tq, Tk, causal;
   float scale;
   unsigned *status;
+  // Optional per-sequence lengths (device arrays of B ints) and per-sequence
+  // 3-D maps (D, length, H) of Q, K, V (device array of 3*B maps).
+  const int *q_lens = nullptr, *kv_lens = nullptr;
+  const CUtensorMap *maps = nullptr;
 };
 // tmQ/tmK/tmV: 4-D maps (D=128, T, H, B), bf16, box (64, 128, 1, 1), 128-byte swizzle.
 int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,

@@ -155,6 +155,41 @@ GMLA_API gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_str
                                 float *lse, float *weights, gmla_stream_t stream);
 
 /*
+ * gmla_attend_prefill_varlen -- gmla_attend_prefill over a padded batch whose
+ * sequences have their own query and key counts: the two-dimensional padding
+ * mask of the "Kimi K2 - Construct causal mask" page in length form, with the
+ * causal mask applied per sequence at that page's positions (queries
+ * continue after the sequence's past length).
+ *
+ *  Sequence b has q_lens[b] query rows (rows 0..q_lens[b]-1 of Q) and
+ *  kv_lens[b] keys (rows 0..kv_lens[b]-1 of K and V); its query t sits at
+ *  position kv_lens[b] - q_lens[b] + t.  Rows past a length are never read as
+ *  data (they may hold anything, NaN included) and output rows t >= q_lens[b]
+ *  of O and lse are left untouched.
+ *  q_lens, kv_lens  HOST arrays of B lengths, 0 <= q_lens[b] <= kv_lens[b],
+ *          q_lens[b] <= Tq_max, 1 <= kv_lens[b] <= Tk_max; read during the
+ *          call only.
+ *  Q, O    [B, Tq_max, H, D_h]; K, V [B, Tk_max, H, D_h]; G [B, Tq_max, H*D_h];
+ *          lse [B, H, Tq_max] -- as for gmla_attend_prefill (strides in
+ *          elements, last dimension contiguous).  No debug weights.
+ *  workspace >= gmla_attend_prefill_varlen_workspace_size(B) bytes, 16-byte
+ *          aligned; it receives three tensor maps and two lengths per
+ *          sequence, copied from the host on `stream` before the launch.
+ * Errors: GMLA_ERR_ARG for null pointers, lengths outside those bounds, bad
+ * strides or alignment; GMLA_ERR_UNSUPPORTED for D_h != 128;
+ * GMLA_ERR_WORKSPACE for a short workspace.
+ */
+GMLA_API gmla_status gmla_attend_prefill_varlen(const gmla_bf16 *Q, const int64_t q_strides[3],
+                                               const gmla_bf16 *K, const int64_t k_strides[3],
+                                               const gmla_bf16 *V, const int64_t v_strides[3], int64_t B,
+                                               int64_t H, int64_t Tq_max, int64_t Tk_max, int64_t D_h,
+                                               const int64_t *q_lens, const int64_t *kv_lens, int causal,
+                                               float scale, const gmla_bf16 *G, gmla_bf16 *O,
+                                               const int64_t o_strides[3], float *lse, void *workspace,
+                                               size_t workspace_bytes, gmla_stream_t stream);
+GMLA_API size_t gmla_attend_prefill_varlen_workspace_size(int64_t B);
+
+/*
  * gmla_attend_decode -- one new query per sequence over the latent cache.
  * Same mathematics as gmla_attend_prefill with Tq = 1 over K = C W_k^T and
  * V = C W_v^T ("Gated MLA" page, "Start from familiar attention"), evaluated

@@ -100,6 +100,13 @@ def test_host_validation_without_gpu(gmla):
     assert LV(fake, fake, 2, 100, lens, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 16, None) == 5
     assert L.gmla_attend_decode_varlen_workspace_size(2, 100, 2, 64) > L.gmla_attend_decode_workspace_size(2, 100, 2,
                                                                                                           64)
+    # varlen prefill: q_len > kv_len, kv_len 0, a short workspace
+    PV = L.gmla_attend_prefill_varlen
+    ql, kl = (ctypes.c_int64 * 2)(10, 20), (ctypes.c_int64 * 2)(20, 20)
+    qbad, kbad = (ctypes.c_int64 * 2)(21, 20), (ctypes.c_int64 * 2)(20, 0)
+    for qq, kk, ws, code in ((qbad, kl, 1 << 20, 1), (ql, kbad, 1 << 20, 1), (ql, kl, 8, 5)):
+        assert PV(fake, s, fake, s, fake, s, 2, 2, 300, 300, 128, qq, kk, 1, 0.0, None, fake, s, None, fake, ws,
+                  None) == code
     # expand_kv: range past the cache, no output, d_model not a multiple of 128
     assert L.gmla_expand_kv(fake, 2, 100, 50, 51, 64, fake, fake, 256, fake, fake, None) == 1
     assert L.gmla_expand_kv(fake, 2, 100, 0, 10, 64, fake, fake, 256, None, None, None) == 1

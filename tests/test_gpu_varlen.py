@@ -96,3 +96,83 @@ def test_decode_varlen_full_size_sampled(g):
                                 heads=[(0, h)])
         sl = slice(h * 128, (h + 1) * 128)
         assert_parity(got[b, sl], ref[0, sl], f"varlen full-size b={b} h={h} length {n}")
+
+
+def _prefill_varlen_inputs(seed, B, Tq, Tk, H, q_lens, kv_lens):
+    from synth_inputs import prefill_qkv
+    inp = prefill_qkv(seed, B, Tq, H, Tk=Tk, gate=True)
+    dirty = {k: v.copy() for k, v in inp.items()}
+    for b in range(B):
+        dirty["Q"][b, q_lens[b]:] = 0x7FC0  # bfloat16 quiet NaN in the padding
+        dirty["K"][b, kv_lens[b]:] = 0x7FC0
+        dirty["V"][b, kv_lens[b]:] = 0x7FC0
+    return inp, dirty
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_varlen_matches_oracle_per_sequence(g, causal):
+    """Padded prefill batch: a full square sequence, an empty one, a 37-row chunk
+    continuing 483 cached keys, a single tile, and a 1-row chunk over 257 keys.
+    NaN padding; output and lse rows past each q_len stay untouched."""
+    B, H, Tq, Tk = 5, 2, 300, 520
+    q_lens = [300, 0, 37, 129, 1]
+    kv_lens = [300, 5, 520, 129, 257]
+    inp, dirty = _prefill_varlen_inputs(1301, B, Tq, Tk, H, q_lens, kv_lens)
+    Q, K, V, G = (to_dev(dirty[k]) for k in ("Q", "K", "V", "G"))
+    sentinel = 0x1234
+    O = torch.from_numpy(np.full((B, Tq, H, 128), sentinel, dtype=np.int16)).view(torch.bfloat16).cuda()
+    lse = torch.full((B, H, Tq), float("nan"), device="cuda")
+    work = torch.empty(g.gmla_attend_prefill_varlen_workspace_size(B), dtype=torch.uint8, device="cuda")
+    g.gmla_attend_prefill_varlen(Q, K, V, O, q_lens, kv_lens, causal=causal, G=G, lse=lse, workspace=work)
+    g.gmla_get_device_status()
+    got, ob, lg = f64(O), bits(O), f64(lse)
+    for b in range(B):
+        q, kv = q_lens[b], kv_lens[b]
+        assert np.all(ob[b, q:] == sentinel), f"sequence {b}: padded output rows were written"
+        assert np.all(np.isnan(lg[b, :, q:]))
+        if q == 0:
+            continue
+        ref, lref = orc.attention(inp["Q"][b:b + 1, :q], inp["K"][b:b + 1, :kv], inp["V"][b:b + 1, :kv],
+                                  causal=causal, want_lse=True)
+        ref = orc.gate(ref.reshape(1, q, -1), inp["G"][b:b + 1, :q]).reshape(ref.shape)
+        assert_parity(got[b:b + 1, :q], ref, f"varlen prefill sequence {b} (q={q}, kv={kv})")
+        np.testing.assert_allclose(lg[b:b + 1, :, :q], lref, atol=5e-4)
+
+
+def test_prefill_varlen_equal_lengths_equals_uniform(g):
+    """All lengths at their maxima: the same kernel as gmla_attend_prefill reading the
+    same data through per-sequence maps, so the outputs match bit for bit."""
+    B, H, Tq, Tk = 2, 3, 300, 333
+    from synth_inputs import prefill_qkv
+    inp = prefill_qkv(1302, B, Tq, H, Tk=Tk, gate=True)
+    Q, K, V, G = (to_dev(inp[k]) for k in ("Q", "K", "V", "G"))
+    O1, O2 = torch.empty_like(Q), torch.empty_like(Q)
+    g.gmla_attend_prefill(Q, K, V, O1, G=G)
+    work = torch.empty(g.gmla_attend_prefill_varlen_workspace_size(B), dtype=torch.uint8, device="cuda")
+    g.gmla_attend_prefill_varlen(Q, K, V, O2, [Tq] * B, [Tk] * B, G=G, workspace=work)
+    g.gmla_get_device_status()
+    assert np.array_equal(bits(O1), bits(O2))
+
+
+def test_prefill_varlen_large_sampled(g):
+    """Mixed lengths up to 8192 (a full square sequence, a 1000-row chunk over 8192
+    keys, a 4096-row chunk over 6000 keys), sampled rows per sequence and head."""
+    B, H, Tq, Tk = 3, 4, 8192, 8192
+    q_lens, kv_lens = [8192, 1000, 4096], [8192, 8192, 6000]
+    inp, dirty = _prefill_varlen_inputs(1303, B, Tq, Tk, H, q_lens, kv_lens)
+    Q, K, V = (to_dev(dirty[k]) for k in ("Q", "K", "V"))
+    O = torch.zeros_like(Q)
+    work = torch.empty(g.gmla_attend_prefill_varlen_workspace_size(B), dtype=torch.uint8, device="cuda")
+    g.gmla_attend_prefill_varlen(Q, K, V, O, q_lens, kv_lens, workspace=work)
+    g.gmla_get_device_status()
+    got = f64(O)
+    rng = np.random.default_rng(1303)
+    for b in range(B):
+        q, kv = q_lens[b], kv_lens[b]
+        ts = sorted(set([0, 1, 127, 128, q // 2, q - 1] + list(rng.integers(0, q, 4))))
+        for h in (0, H - 1):
+            sl = lambda k, n: inp[k][b:b + 1, :n, h:h + 1]
+            ref = orc.attention(sl("Q", q), sl("K", kv), sl("V", kv), rows=[(0, 0, t) for t in ts])
+            assert_parity(np.stack([got[b, t, h] for t in ts]), np.stack([ref[0, t, 0] for t in ts]),
+                          f"varlen prefill b={b} h={h}")
+    assert np.all(np.isfinite(got))
