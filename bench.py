@@ -48,6 +48,12 @@ SWEEP_T = (8192, 131072, 1048576)
 SWEEP_H = 8
 SWEEP_B = 4
 SWEEP_PAGE = {"dot_products_per_head": (3.2e7, 8.2e9, 5.2e11), "kv_cache": (1, 16, 128)}
+# --workload varlen: a padded prefill batch of chunks continuing differently cached sequences
+# (per-sequence query / key lengths) and a decode batch with per-sequence cache lengths
+VL_H = 32
+VL_Q = (8192, 4096, 2048, 1024, 8192, 512, 3000, 100)
+VL_KV = (8192, 8192, 6000, 1024, 8192, 4096, 3000, 5000)
+VL_DEC_B, VL_DEC_LMAX = 32, 131072
 
 
 def prefill_flops(B=P_B, H=P_H, T=P_T):
@@ -77,7 +83,7 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 # from one ncu capture each (profiles/).  Reported only while the kernel source is the one that
 # was captured (sha1 of the file); any change makes it null until the next capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill.cu": {"sha1": "bb501558ebeb19bc821a219788ea5b8e5481a8d1", "bytes": 604.078848e6 + 185.454080e6,
+    "attn_prefill.cu": {"sha1": "ffe545376afcfed7e56882a64169aa1db2a810c1", "bytes": 604.147456e6 + 183.511808e6,
                         "how": "ncu capture at the timed size (B=1 H=96 T=8192)"},
     "attn_latent_tc.cu": {"sha1": "364762a2d84494c68f2ebb53fa6143c2fc15edc0", "bytes": 544.323328e6 * 8 + 32.472832e6,
                           "how": "ncu capture of latent_decode_kernel at L=16384, reads scaled x8 to L=131072 (cache "
@@ -423,6 +429,73 @@ def timed(fn_list, steps, world):
     return total, per
 
 
+def run_varlen(args, rank, world, local, peaks):
+    """Variable-length batches: gmla_attend_prefill_varlen over VL_Q / VL_KV (H = VL_H;
+    flops count each sequence's own causal pairs) and gmla_attend_decode_varlen at
+    B = VL_DEC_B with seeded lengths in 1..VL_DEC_LMAX (bytes count visible latents)."""
+    import torch
+
+    import causal_head_latent_b200 as g
+    from synth_inputs import Draw, prefill_qkv
+
+    B = len(VL_Q)
+    Tq, Tk = max(VL_Q), max(VL_KV)
+    inp = prefill_qkv(1401, B, Tq, VL_H, Tk=Tk)
+    Q, K, V = (dev(inp[k]) for k in ("Q", "K", "V"))
+    del inp
+    O = torch.empty_like(Q)
+    wsp = torch.empty(g.gmla_attend_prefill_varlen_workspace_size(B), dtype=torch.uint8, device="cuda")
+    pairs = sum(q * (kv - q) + q * (q + 1) // 2 for q, kv in zip(VL_Q, VL_KV))
+    pf = 4.0 * D * VL_H * pairs
+
+    dr = Draw(1402)
+    lens = [int(x) for x in np.random.default_rng(1402).integers(1, VL_DEC_LMAX + 1, VL_DEC_B)]
+    H, d = DM // D, DM
+    q = dev(dr.normal((VL_DEC_B, d)))
+    Wk = dev(dr.normal((d, DC), 1 / np.sqrt(DC)))
+    Wv = dev(dr.normal((d, DC), 1 / np.sqrt(DC)))
+    C = dev(dr.normal((VL_DEC_B, VL_DEC_LMAX, DC)))
+    Od = torch.empty(VL_DEC_B, d, dtype=torch.bfloat16, device="cuda")
+    wsd = torch.empty(g.gmla_attend_decode_varlen_workspace_size(VL_DEC_B, VL_DEC_LMAX, H, DC), dtype=torch.uint8,
+                      device="cuda")
+    db = 2.0 * (sum(lens) * DC + 2 * d * DC + 2 * VL_DEC_B * d)
+
+    fp = lambda: g.gmla_attend_prefill_varlen(Q, K, V, O, VL_Q, VL_KV, workspace=wsp)
+    fd = lambda: g.gmla_attend_decode_varlen(q, C, lens, Wk, Wv, Od, H, workspace=wsd)
+    for _ in range(args.warmup):
+        fp()
+        fd()
+    g.gmla_get_device_status()
+    clk = ClockSampler(local)
+    clk.start()
+    total, per = timed([fp, fd], args.steps, world)
+    clocks = clk.stop()
+    g.gmla_get_device_status()
+    total = max_over_ranks(total, world)
+    p_ms = max_over_ranks(per[0], world) / args.steps
+    d_ms = max_over_ranks(per[1], world) / args.steps
+    p_tf = pf / (p_ms / 1e3) / 1e12
+    d_gbs = db / (d_ms / 1e3) / 1e9
+    line = {"metric": "variable-length batches: padded prefill attention TFLOP/s (per-sequence causal pairs) and "
+                      "per-sequence-length latent decode GB/s",
+            "value": p_tf, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"gmla_attend_prefill_varlen B={B} H={VL_H} D_h={D} q_lens={list(VL_Q)} "
+                                   f"kv_lens={list(VL_KV)} + gmla_attend_decode_varlen B={VL_DEC_B} H=96 d_c={DC} "
+                                   f"lengths seeded in 1..{VL_DEC_LMAX} (sum {sum(lens)})",
+                       "l2": "inputs larger than L2; no flush"},
+            "clocks": clocks, "gpu_launches": 4 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": p_tf, "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": p_tf / peaks["bf16_tflops_sustained"], "traffic": None},
+            "decode": {"value": d_gbs, "unit": "GB/s", "ms_per_step": d_ms,
+                       "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": d_gbs / peaks["hbm_gbs"], "traffic": None}},
+            "prefill_ms": p_ms}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_sweep(args, rank, world, local, peaks):
     """Long-context sweep: causal prefill attention (B=1, SWEEP_H heads) and latent-cache
     decode (B=SWEEP_B, 96 heads, d_c=512) at each length of SWEEP_T, each timed with CUDA
@@ -507,7 +580,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--parts", default="all", choices=["all", "prefill", "decode"])
-    ap.add_argument("--workload", default="step", choices=["step", "layer", "sweep"])
+    ap.add_argument("--workload", default="step", choices=["step", "layer", "sweep", "varlen"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--dec-L", type=int, default=DEC_L,
@@ -529,6 +602,9 @@ def main():
 
     if args.workload == "sweep":
         run_sweep(args, rank, world, local, peaks)
+        return
+    if args.workload == "varlen":
+        run_varlen(args, rank, world, local, peaks)
         return
 
     if args.workload == "layer":
