@@ -28,17 +28,20 @@
 // Hence 48-key tiles: an 18-chunk latent ring (2.25 tiles) lets the loads of
 // tile j stream while tiles j-1 and j-2 are still in use; S is double-
 // buffered in TMEM so the score MMAs of the next tile never wait for the
-// softmax; the value MMAs of tile j-1 sit between the two parts of the score
-// MMAs of tile j, late enough for the softmax of tile j-1 and early enough
-// to release ring slots for tile j+2; and the ring moves in chunk pairs, so a
-// tile costs the MMA thread two data waits, one softmax wait and three
-// commits.
+// softmax; the score and value MMAs come from two threads, so the value MMAs
+// of a tile go out as soon as its probabilities are ready (releasing ring
+// slots for tile j+2 early) while score MMAs keep the pipe busy; and the ring
+// moves in chunk pairs, so a tile costs the score thread three waits and one
+// commit and the value thread one wait and two commits.
 //
 //   warp 0      TMA producer: q~ once, then the latents in 64-column chunks
 //               (6 KB: 48 keys x 64 d_c) through the ring
-//   warp 1      TMEM owner, MMA issuer (one thread)
+//   warp 1      TMEM owner; issues the score MMAs (one thread)
 //   warps 2..5  softmax, one head per TMEM lane; lazy rescale of acc^T when a
 //               head's running max grows by more than 2^8; partial-state store
+//   warp 6      issues the value MMAs (one thread)
+// Two issuing threads: a wait of one (for data, for the softmax) does not
+// leave the tensor pipe idle while the other has MMAs to issue.
 //
 // q~ in shared memory: eight 64-column chunks of 96 rows (12 KB each) placed
 // 12 KB apart.  The score MMA reads 128-row A tiles, so rows 96..127 of chunk
@@ -56,7 +59,7 @@ namespace latent_tc {
 
 constexpr int HMAX = 96;
 constexpr int KT = 48;                    // keys per tile: N of the score product
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 224;
 constexpr int NCHUNK = 8;                 // 64-wide d_c chunks per tile (d_c <= 512)
 constexpr int QCHUNK = HMAX * 128;        // 12 KB: one d_c chunk of q~ for 96 heads
 constexpr int Q_BYTES = NCHUNK * QCHUNK;  // 96 KB
@@ -157,10 +160,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *full_l = full_e + NTB;       // [NTB]: the remaining pairs of tile j landed
   uint64_t *rel = full_l + NTB;          // [NTB][2]: pairs 2h, 2h+1 of tile j released
   uint64_t *s_full = rel + 2 * NTB;      // [2]
-  uint64_t *p_full = s_full + 2;
+  uint64_t *s_free = s_full + 2;         // [2]: the softmax has read S buffer i
+  uint64_t *p_full = s_free + 2;
   uint64_t *acc_done = p_full + 1;
-  uint64_t *mma_idle = acc_done + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_idle + 1);
+  uint64_t *mma_idle = acc_done + 1;     // [2]: one per issuing thread
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_idle + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int b = blockIdx.x / p.n_splits;
@@ -188,10 +192,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&rel[2 * t], 1);
       mbar_init(&rel[2 * t + 1], 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&mma_idle[i], 1);
+    }
     mbar_init(p_full, 4);
     mbar_init(acc_done, 1);
-    mbar_init(mma_idle, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -249,13 +256,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // ---------------------------------------------------------------- score MMAs
       constexpr uint32_t idS = idesc_bf16_f32(128, KT, false, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(128, HMAX, true, false);
-      const uint32_t aq = smem_u32(sq), ac = smem_u32(sc), ap = smem_u32(sp);
-      // Score MMAs of chunk pairs [q0, q1) of tile j into S buffer j&1.  That
-      // buffer was last read by the softmax of tile j-2, whose p_full this
-      // thread waited for (followed by tcgen05.fence::after_thread_sync)
-      // before the value MMAs of tile j-2.
+      const uint32_t aq = smem_u32(sq), ac = smem_u32(sc);
+      // Score MMAs of chunk pairs [q0, q1) of tile j into S buffer j&1.
       auto score_pairs = [&](int j, int q0, int q1) -> bool {
         const uint32_t dS = tmem + TM_S + (j & 1) * 64;
         // TMA completion on the mbarrier orders the copies before the MMA's reads
@@ -273,36 +277,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return true;
       };
       bool ok = mbar_wait(bar_q, 0, p.status);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles && !score_pairs(j, 0, NEARLY_PAIRS)) break;
-        if (j >= 1) {
-          const int jp = j - 1;
-          if (!mbar_wait_relaxed(p_full, jp & 1, p.status)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
-            const int g = jp * NPT + blk;
-            const uint32_t cst = ac + (g % NPAIR) * 2 * CCHUNK;
-#pragma unroll
-            for (int ks = 0; ks < KT / 16; ++ks)
-              umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
-                           sdesc_sw128(ap + ks * 32, 16, 1024), idPV, (jp > 0 || ks > 0) ? 1u : 0u);
-            if (blk & 1) umma_commit(&rel[2 * (jp % NTB) + (blk >> 1)]);
-          }
-          if (jp == n_tiles - 1) umma_commit(acc_done);
-        }
-        if (j < n_tiles) {
-          if (!score_pairs(j, NEARLY_PAIRS, NPT)) break;
-          // Arrives once S_j and everything issued before it -- the value
-          // MMAs of tile j-1 among them -- have completed, so the softmax of
-          // tile j may rewrite P^T and rescale acc^T.
-          umma_commit(&s_full[j & 1]);
-        }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        // S buffer j&1 was last read by the softmax of tile j-2
+        if (j >= 2 && !mbar_wait_relaxed(&s_free[j & 1], ((j - 2) >> 1) & 1, p.status)) break;
+        tc_fence_after();
+        if (!score_pairs(j, 0, NEARLY_PAIRS) || !score_pairs(j, NEARLY_PAIRS, NPT)) break;
+        umma_commit(&s_full[j & 1]);
       }
-      // Every path: wait until the MMAs issued so far have finished before
-      // the CTA releases TMEM.
-      umma_commit(mma_idle);
-      mbar_wait_limit(mma_idle, 0, p.status, kDrainLimitNs);
+      // Every path: wait until this thread's MMAs have finished before the
+      // CTA releases TMEM.
+      umma_commit(&mma_idle[0]);
+      mbar_wait_limit(&mma_idle[0], 0, p.status, kDrainLimitNs);
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- value MMAs
+      constexpr uint32_t idPV = idesc_bf16_f32(128, HMAX, true, false);
+      const uint32_t ac = smem_u32(sc), ap = smem_u32(sp);
+      for (int j = 0; j < n_tiles; ++j) {
+        if (!mbar_wait_relaxed(p_full, j & 1, p.status)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          const int g = j * NPT + blk;
+          const uint32_t cst = ac + (g % NPAIR) * 2 * CCHUNK;
+#pragma unroll
+          for (int ks = 0; ks < KT / 16; ++ks)
+            umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
+                         sdesc_sw128(ap + ks * 32, 16, 1024), idPV, (j > 0 || ks > 0) ? 1u : 0u);
+          // rel[.][1] also tells the softmax of tile j+1 that P^T and acc^T are free
+          if (blk & 1) umma_commit(&rel[2 * (j % NTB) + (blk >> 1)]);
+        }
+        if (j == n_tiles - 1) umma_commit(acc_done);
+      }
+      umma_commit(&mma_idle[1]);
+      mbar_wait_limit(&mma_idle[1], 0, p.status, kDrainLimitNs);
     }
   } else {
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
@@ -328,6 +337,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < KT; ++c) x[c] = -INFINITY;
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[sb]);
       }
       const int k0 = k_begin + j * KT;
       float mx = -INFINITY;
@@ -342,8 +354,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (k0 + c < k_end) wrow[k0 + c] = x[c];
       }
       const bool need = head_ok && mx > m_used + kRescaleThreshold;
-      if (bar_or(1, 128, need || !got)) {
-        if (bar_or(1, 128, !got)) {  // a wait gave up: every softmax thread leaves together
+      // P^T and acc^T are free once the value MMAs of tile j-1 have completed
+      bool ready = got;
+      if (got && j >= 1) {
+        const int jp = j - 1;
+        ready = __all_sync(0xffffffffu, mbar_wait(&rel[2 * (jp % NTB) + 1], (jp / NTB) & 1, p.status));
+        tc_fence_after();
+      }
+      if (bar_or(1, 128, need || !ready)) {
+        if (bar_or(1, 128, !ready)) {  // a wait gave up: every softmax thread leaves together
           ok = false;
           break;
         }
@@ -357,7 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bar_sync(1, 128);  // alpha_s complete
         if (j > 0) {
           // acc^T lanes are d_c rows, columns are heads: scale column h by
-          // alpha_s[h].  The value MMAs of tile j-1 have completed (s_full).
+          // alpha_s[h].  The value MMAs of tile j-1 have completed (rel).
 #pragma unroll 1
           for (int blk = 0; blk < 4; ++blk) {
 #pragma unroll 1
@@ -383,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         pk[c / 2] = pack_bf16x2(p0, p1);
       }
       l += rs;
-      // P^T row h (free: the value MMAs of tile j-1 completed before s_full)
+      // P^T row h (free: the value MMAs of tile j-1 have completed)
       if (active) {
 #pragma unroll
         for (int u = 0; u < KT / 8; ++u)
@@ -435,7 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 size_t smem_bytes() {
-  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 4 * NTB + 5) + 16;
+  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 4 * NTB + 9) + 16;
 }
 
 }  // namespace latent_tc
