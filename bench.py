@@ -85,7 +85,7 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 PROFILED_TRAFFIC = {
     "attn_prefill.cu": {"sha1": "ffe545376afcfed7e56882a64169aa1db2a810c1", "bytes": 604.147456e6 + 183.511808e6,
                         "how": "ncu capture at the timed size (B=1 H=96 T=8192)"},
-    "attn_latent_tc.cu": {"sha1": "364762a2d84494c68f2ebb53fa6143c2fc15edc0", "bytes": 544.323328e6 * 8 + 32.472832e6,
+    "attn_latent_tc.cu": {"sha1": "4e8f5fb90ca5916411bfc57aec6f7184683f8cb9", "bytes": 543.840256e6 * 8 + 32.554752e6,
                           "how": "ncu capture of latent_decode_kernel at L=16384, reads scaled x8 to L=131072 (cache "
                                  "traffic grows with L), partial-state writes unscaled"},
 }
