@@ -16,6 +16,21 @@
  * Softmax over keys") and no positional encoding.  The latent C is the only
  * cached tensor.
  *
+ * Entry points
+ * ------------
+ *  gmla_latent_project       projections [Q | G | C] = X [W_q; W_g; W_c]^T (C into
+ *                            the cache rows) and optionally K, V of those rows
+ *  gmla_expand_kv            K, V of any range of cached latent rows
+ *  gmla_attend_prefill       causal (or full) attention over explicit Q, K, V
+ *  gmla_attend_prefill_varlen  the same over a padded batch with per-sequence
+ *                            query / key lengths
+ *  gmla_attend_decode        one new query per sequence over the latent cache
+ *  gmla_attend_decode_varlen   the same with per-sequence cache lengths
+ *  gmla_attend_decode_noalloc  gmla_attend_decode without a caller workspace
+ *  gmla_gate_out             the output projection Y = O W_o^T
+ *  gmla_get_device_status, gmla_selftest_wait_timeout, gmla_status_string,
+ *  gmla_version, and a *_workspace_size query per call that needs scratch.
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Every tensor is bfloat16 (gmla_bf16 holds the raw 16-bit pattern) unless
