@@ -101,16 +101,34 @@ __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
     if (P.lse2) P.lse2[(size_t)b * P.H + h] = M + __log2f(Lsum);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < nb * dc; i += CT) {
-    const int bb = i / dc, c = i % dc;
-    const float *acc = P.part_acc + ((size_t)(b0 + bb) * P.H + h) * dc + c;
-    const size_t split_stride = (size_t)P.B * P.H * dc;
-    float a = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float ws = wsp[bb * S + s];
-      if (ws != 0.f) a = fmaf(ws, acc[s * split_stride], a);  // an empty split left no acc
+  // c^ = sum_s w_s acc_s: four latent columns per thread (16-byte loads) and
+  // eight splits' loads in flight before their multiply-adds.
+  {
+    const size_t split_stride4 = (size_t)P.B * P.H * dc / 4;
+    for (int i4 = threadIdx.x; i4 < nb * dc / 4; i4 += CT) {
+      const int bb = (i4 * 4) / dc, c = (i4 * 4) % dc;
+      const float4 *src = reinterpret_cast<const float4 *>(P.part_acc + ((size_t)(b0 + bb) * P.H + h) * dc + c);
+      const float *w = wsp + bb * S;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < S; s0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          // an empty split (weight 0) left no acc: never read it
+          v[u] = (s0 + u < S && w[s0 + u] != 0.f) ? src[(size_t)(s0 + u) * split_stride4]
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float ws = (s0 + u < S) ? w[s0 + u] : 0.f;
+          a.x = fmaf(ws, v[u].x, a.x);
+          a.y = fmaf(ws, v[u].y, a.y);
+          a.z = fmaf(ws, v[u].z, a.z);
+          a.w = fmaf(ws, v[u].w, a.w);
+        }
+      }
+      *reinterpret_cast<float4 *>(chat + bb * dc + c) = a;
     }
-    chat[i] = a;
   }
   __syncthreads();
   const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
