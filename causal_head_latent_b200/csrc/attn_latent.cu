@@ -48,12 +48,23 @@ __global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict_
     float acc[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < HD; ++d) {
-      const float w = bf16_to_f32(Wk[((size_t)h * HD + d) * dc + c]);
+    // four rows d of W_k per step, so q is read from shared memory as one
+    // 16-byte broadcast per sequence instead of four
+#pragma unroll 1
+    for (int d = 0; d < HD; d += 4) {
+      float w[4];
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < nb) acc[j] = fmaf(qs[(b0 + j) * HD + d], w, acc[j]);
+      for (int e = 0; e < 4; ++e) w[e] = bf16_to_f32(Wk[((size_t)h * HD + d + e) * dc + c]);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < nb) {
+          const float4 q4 = *reinterpret_cast<const float4 *>(qs + (b0 + j) * HD + d);
+          acc[j] = fmaf(q4.x, w[0], acc[j]);
+          acc[j] = fmaf(q4.y, w[1], acc[j]);
+          acc[j] = fmaf(q4.z, w[2], acc[j]);
+          acc[j] = fmaf(q4.w, w[3], acc[j]);
+        }
+      }
     }
 #pragma unroll
     for (int j = 0; j < 32; ++j)
