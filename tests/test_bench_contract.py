@@ -1,0 +1,70 @@
+"""bench.py without a GPU: the reference arm (the float64 oracle timed on the
+host) prints one JSON line with the contract's keys, ranks other than 0 print
+nothing, and the workload arithmetic matches the figures the timed
+configurations are quoted with."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+from tests.conftest import ROOT
+
+BENCH = os.path.join(ROOT, "bench.py")
+
+
+def _load_bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", BENCH)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _run(args, env_extra=None, timeout=300):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, BENCH] + args, cwd=ROOT, env=env, capture_output=True, text=True,
+                          timeout=timeout)
+
+
+def test_reference_arm_json_line():
+    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference"
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert line["config"]["workload"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_are_silent():
+    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "0", "--gpus", "2"],
+             {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+
+
+def test_workload_arithmetic():
+    b = _load_bench()
+    # causal pairs T(T+1)/2 per head, 4*D flop per pair (QK^T and PV): 1.6495e12 at B=1, H=96, T=8192
+    assert b.prefill_flops(1, 96, 8192) == pytest.approx(1.6495e12, rel=1e-4)
+    # the decode streams every visible latent once: B*L*d_c*2 bytes = 4.295e9 at B=32, L=131072
+    latents = 32 * 131072 * 512 * 2
+    assert latents == pytest.approx(4.295e9, rel=1e-3)
+    extra = b.decode_bytes(32, 131072) - latents
+    assert 0 < extra < 0.02 * latents  # W_k, W_v, q, G and O on top of the cache
+    # the sweep's lengths are the cost table's, whose dot-product orders they reproduce
+    assert b.SWEEP_T == (8192, 131072, 1048576)
+    for t, order in zip(b.SWEEP_T, b.SWEEP_PAGE["dot_products_per_head"]):
+        assert t * (t + 1) / 2 == pytest.approx(order, rel=0.06)
