@@ -468,11 +468,7 @@ int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint
   using namespace latent_tc;
   auto kern = latent_decode_kernel;
   const size_t smem = smem_bytes();
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return -1;
-    configured = true;
-  }
+  if (!set_smem_limit_once(reinterpret_cast<const void *>(kern), (int)smem, kSmemLatentTc)) return -1;
   Params p;
   p.C = C;
   p.Lmax = Lmax;

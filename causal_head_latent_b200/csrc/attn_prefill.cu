@@ -386,13 +386,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
                         const PrefillArgs &a, cudaStream_t stream) {
   using namespace prefill;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  if (!set_smem_limit_once(reinterpret_cast<const void *>(attn_prefill_kernel), (int)kSmemBytes, kSmemPrefill))
+    return -1;
   Params p;
   p.G = a.G;
   p.O = a.O;

@@ -194,13 +194,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &a, cudaStream_t stream) {
   using namespace gemm;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  if (!set_smem_limit_once(reinterpret_cast<const void *>(gemm_kernel), (int)kSmemBytes, kSmemGemm)) return -1;
   Params P;
   P.g = a;
   P.m_tiles_per_b = (a.a_rows + BM - 1) / BM;

@@ -48,6 +48,17 @@ int num_sms() {
   return (d >= 0 && d < kMaxDevices && g_num_sms[d] > 0) ? g_num_sms[d] : 148;
 }
 
+bool set_smem_limit_once(const void *kernel, int bytes, SmemSlot slot) {
+  static bool done[kSmemSlots][kMaxDevices];
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices || slot < 0 || slot >= kSmemSlots) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (done[slot][d]) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done[slot][d] = true;
+  return true;
+}
+
 static unsigned *status_ptr() {
   const int d = current_device();
   if (!device_setup(d)) return nullptr;
