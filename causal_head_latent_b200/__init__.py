@@ -271,9 +271,9 @@ def gmla_attend_decode_varlen(Q, C, lens, W_k, W_v, O, num_heads, scale=0.0, G=N
     H = int(num_heads)
     D = d // H
     _, Lmax, d_c = C.shape
-    lens_arr = (ctypes.c_int64 * B)(*[int(x) for x in lens])
     if len(lens) != B:
         raise ValueError("lens needs one length per sequence")
+    lens_arr = (ctypes.c_int64 * B)(*[int(x) for x in lens])
     wp, wb = _ws(workspace)
     code = lib.gmla_attend_decode_varlen(_ptr(Q), _ptr(C), B, Lmax, ctypes.cast(lens_arr, _p), H, D, d_c, _ptr(W_k),
                                          _ptr(W_v), float(scale), _ptr(G), _ptr(O), _ptr(weights), wp, wb,
