@@ -107,6 +107,14 @@ def test_host_validation_without_gpu(gmla):
     for qq, kk, ws, code in ((qbad, kl, 1 << 20, 1), (ql, kbad, 1 << 20, 1), (ql, kl, 8, 5)):
         assert PV(fake, s, fake, s, fake, s, 2, 2, 300, 300, 128, qq, kk, 1, 0.0, None, fake, s, None, fake, ws,
                   None) == code
+    # varlen prefill: misaligned workspace; head width other than 128
+    assert PV(fake, s, fake, s, fake, s, 2, 2, 300, 300, 128, ql, kl, 1, 0.0, None, fake, s, None, fake + 8, 1 << 20,
+              None) == 1
+    assert PV(fake, s, fake, s, fake, s, 2, 2, 300, 300, 64, ql, kl, 1, 0.0, None, fake, s, None, fake, 1 << 20,
+              None) == 2
+    # varlen decode: more than 96 heads, d_c not a multiple of 64
+    assert LV(fake, fake, 2, 100, lens, 97, 128, 64, fake, fake, 0.0, None, fake, None, fake, 1 << 30, None) == 2
+    assert LV(fake, fake, 2, 100, lens, 2, 128, 96, fake, fake, 0.0, None, fake, None, fake, 1 << 30, None) == 2
     # expand_kv: range past the cache, no output, d_model not a multiple of 128
     assert L.gmla_expand_kv(fake, 2, 100, 50, 51, 64, fake, fake, 256, fake, fake, None) == 1
     assert L.gmla_expand_kv(fake, 2, 100, 0, 10, 64, fake, fake, 256, None, None, None) == 1
