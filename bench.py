@@ -258,11 +258,8 @@ class DecodePart:
         self.O = torch.empty(DEC_B, DM, dtype=torch.bfloat16, device="cuda")
         self.Y = torch.empty_like(self.O)
         self.Y_host = torch.empty(self.Y.shape, dtype=torch.bfloat16).pin_memory()
-        self.ws_p = torch.empty(max(1, g.gmla_latent_project_workspace_size(DEC_B, 1, DM, DC)), dtype=torch.uint8,
-                                device="cuda")
         self.ws_d = torch.empty(g.gmla_attend_decode_workspace_size(DEC_B, DEC_L, DM // D, DC), dtype=torch.uint8,
                                 device="cuda")
-        self.ws_o = torch.empty(max(1, g.gmla_gate_out_workspace_size(DEC_B, DM)), dtype=torch.uint8, device="cuda")
         self.bytes = decode_bytes()
         self.launches = 6
 
@@ -270,7 +267,7 @@ class DecodePart:
         import causal_head_latent_b200 as g
         W = self.W
         g.gmla_latent_project(self.X, W["W_q"], W["W_g"], W["W_c"], None, None, Q=self.Q, G=self.G, C=self.C,
-                              cache_pos=DEC_L - 1, workspace=self.ws_p)
+                              cache_pos=DEC_L - 1)
 
     def attend(self):
         import causal_head_latent_b200 as g
@@ -279,7 +276,7 @@ class DecodePart:
 
     def out(self):
         import causal_head_latent_b200 as g
-        g.gmla_gate_out(self.O, self.W["W_o"], self.Y, workspace=self.ws_o)
+        g.gmla_gate_out(self.O, self.W["W_o"], self.Y)
 
     def run_e2e(self):
         self.X.copy_(self.X_host, non_blocking=True)

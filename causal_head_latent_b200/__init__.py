@@ -18,10 +18,13 @@ import torch
 
 __all__ = [
     "GmlaError", "lib", "library_path",
-    "gmla_latent_project", "gmla_latent_project_workspace_size",
+    "gmla_latent_project", "gmla_latent_project_heads",
     "gmla_expand_kv", "gmla_attend_prefill", "gmla_attend_prefill_varlen", "gmla_attend_prefill_varlen_workspace_size",
-    "gmla_attend_decode", "gmla_attend_decode_workspace_size",
-    "gmla_gate_out", "gmla_gate_out_workspace_size", "gmla_get_device_status", "gmla_status_string",
+    "gmla_attend_decode", "gmla_attend_decode_workspace_size", "gmla_attend_decode_varlen",
+    "gmla_attend_decode_varlen_workspace_size", "gmla_attend_decode_partial", "gmla_attend_decode_partial_workspace_size",
+    "gmla_decode_combine", "gmla_attend_decode_noalloc", "gmla_attend_decode_noalloc_max_bytes",
+    "gmla_gate_out", "gmla_gate_out_heads", "gmla_gate_out_workspace_size", "gmla_get_device_status",
+    "gmla_selftest_wait_timeout", "gmla_status_string",
     "gmla_version", "STATUS",
 ]
 
@@ -32,7 +35,7 @@ STATUS = {0: "GMLA_OK", 1: "GMLA_ERR_ARG", 2: "GMLA_ERR_UNSUPPORTED", 3: "GMLA_E
           4: "GMLA_ERR_TIMEOUT", 5: "GMLA_ERR_WORKSPACE"}
 
 if not os.path.exists(library_path):
-    raise ImportError(f"libgmla.so not built ({library_path}); run `python -m causal_head_latent_b200.build`")
+    raise ImportError(f"libgmla.so not built ({library_path}); run `python causal_head_latent_b200/build.py`")
 
 lib = ctypes.CDLL(library_path)
 
@@ -43,10 +46,11 @@ _st = ctypes.c_int
 _i64x3 = ctypes.c_int64 * 3
 
 lib.gmla_latent_project.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _i64, _i64,
-                                    _p, _p, _p, _sz, _p]
+                                    _p, _p, _p]
 lib.gmla_latent_project.restype = _st
-lib.gmla_latent_project_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
-lib.gmla_latent_project_workspace_size.restype = _sz
+lib.gmla_latent_project_heads.argtypes = [_p, _i64, _i64, _i64, _i64, _i64, _p, _p, _p, _i64, _p, _p, _p, _p, _p, _i64,
+                                          _i64, _p, _p, _p]
+lib.gmla_latent_project_heads.restype = _st
 lib.gmla_expand_kv.argtypes = [_p, _i64, _i64, _i64, _i64, _i64, _p, _p, _i64, _p, _p, _p]
 lib.gmla_expand_kv.restype = _st
 lib.gmla_attend_prefill.argtypes = [_p, _i64x3, _p, _i64x3, _p, _i64x3, _i64, _i64, _i64, _i64, _i64,
@@ -67,6 +71,13 @@ lib.gmla_attend_decode_varlen.argtypes = [_p, _p, _i64, _i64, _p, _i64, _i64, _i
 lib.gmla_attend_decode_varlen.restype = _st
 lib.gmla_attend_decode_varlen_workspace_size.argtypes = [_i64, _i64, _i64, _i64]
 lib.gmla_attend_decode_varlen_workspace_size.restype = _sz
+lib.gmla_attend_decode_partial.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _p, ctypes.c_float, _p,
+                                           _p, _p, _sz, _p]
+lib.gmla_attend_decode_partial.restype = _st
+lib.gmla_attend_decode_partial_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64]
+lib.gmla_attend_decode_partial_workspace_size.restype = _sz
+lib.gmla_decode_combine.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _p, _p, _p, _p]
+lib.gmla_decode_combine.restype = _st
 lib.gmla_attend_decode_noalloc.argtypes = [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p,
                                            _p, _p, _p]
 lib.gmla_attend_decode_noalloc.restype = _st
@@ -74,6 +85,8 @@ lib.gmla_attend_decode_noalloc_max_bytes.argtypes = []
 lib.gmla_attend_decode_noalloc_max_bytes.restype = _sz
 lib.gmla_gate_out.argtypes = [_p, _p, _p, _i64, _i64, _p, _p, _sz, _p]
 lib.gmla_gate_out.restype = _st
+lib.gmla_gate_out_heads.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p]
+lib.gmla_gate_out_heads.restype = _st
 lib.gmla_gate_out_workspace_size.argtypes = [_i64, _i64]
 lib.gmla_gate_out_workspace_size.restype = _sz
 lib.gmla_get_device_status.argtypes = [_p]
@@ -146,12 +159,8 @@ def gmla_selftest_wait_timeout(milliseconds: int = 20, stream=None) -> int:
     return _check(lib.gmla_selftest_wait_timeout(int(milliseconds), _stream(stream)), "gmla_selftest_wait_timeout")
 
 
-def gmla_latent_project_workspace_size(B, T, d_model, d_c) -> int:
-    return lib.gmla_latent_project_workspace_size(B, T, d_model, d_c)
-
-
 def gmla_latent_project(X, W_q, W_g, W_c, W_k, W_v, Q=None, G=None, C=None, cache_len_max=None, cache_pos=0,
-                        K=None, V=None, workspace=None, stream=None, check=True):
+                        K=None, V=None, stream=None, check=True):
     """X [B, T, d_model]; C [B, cache_len_max, d_c] (rows cache_pos..cache_pos+T-1 written)."""
     for n, t in (("X", X), ("W_q", W_q), ("W_g", W_g), ("W_c", W_c), ("W_k", W_k), ("W_v", W_v),
                  ("Q", Q), ("G", G), ("C", C), ("K", K), ("V", V)):
@@ -160,11 +169,27 @@ def gmla_latent_project(X, W_q, W_g, W_c, W_k, W_v, Q=None, G=None, C=None, cach
     d_c = W_c.shape[0] if W_c is not None else (C.shape[-1] if C is not None else 0)
     if cache_len_max is None:
         cache_len_max = C.shape[1] if C is not None else T
-    wp, wb = _ws(workspace)
     code = lib.gmla_latent_project(_ptr(X), B, T, d, _ptr(W_q), _ptr(W_g), _ptr(W_c), d_c, _ptr(W_k), _ptr(W_v),
-                                   _ptr(Q), _ptr(G), _ptr(C), cache_len_max, cache_pos, _ptr(K), _ptr(V), wp, wb,
+                                   _ptr(Q), _ptr(G), _ptr(C), cache_len_max, cache_pos, _ptr(K), _ptr(V),
                                    _stream(stream))
     return _check(code, "gmla_latent_project") if check else code
+
+
+def gmla_latent_project_heads(X, head_begin, head_end, W_q, W_g, W_c, W_k, W_v, Q=None, G=None, C=None,
+                              cache_len_max=None, cache_pos=0, K=None, V=None, stream=None, check=True):
+    """Projections of heads [head_begin, head_end) only: full weights in, Q, G, K, V
+    [B, T, 128*(head_end-head_begin)] out; C (full latent) as gmla_latent_project."""
+    for n, t in (("X", X), ("W_q", W_q), ("W_g", W_g), ("W_c", W_c), ("W_k", W_k), ("W_v", W_v),
+                 ("Q", Q), ("G", G), ("C", C), ("K", K), ("V", V)):
+        _bf16(t, n)
+    B, T, d = X.shape
+    d_c = W_c.shape[0] if W_c is not None else (C.shape[-1] if C is not None else 0)
+    if cache_len_max is None:
+        cache_len_max = C.shape[1] if C is not None else T
+    code = lib.gmla_latent_project_heads(_ptr(X), B, T, d, int(head_begin), int(head_end), _ptr(W_q), _ptr(W_g),
+                                         _ptr(W_c), d_c, _ptr(W_k), _ptr(W_v), _ptr(Q), _ptr(G), _ptr(C),
+                                         cache_len_max, cache_pos, _ptr(K), _ptr(V), _stream(stream))
+    return _check(code, "gmla_latent_project_heads") if check else code
 
 
 def gmla_expand_kv(C, row0, rows, W_k=None, W_v=None, K=None, V=None, stream=None, check=True):
@@ -301,12 +326,51 @@ def gmla_attend_decode_noalloc(Q, C, L, W_k, W_v, O, num_heads, scale=0.0, G=Non
     return _check(code, "gmla_attend_decode_noalloc") if check else code
 
 
+def gmla_attend_decode_partial_workspace_size(B, k0, k1, H, d_c) -> int:
+    return lib.gmla_attend_decode_partial_workspace_size(B, k0, k1, H, d_c)
+
+
+def gmla_attend_decode_partial(Q, C, k0, k1, W_k, lse, ctx, num_heads, scale=0.0, workspace=None, stream=None,
+                               check=True):
+    """Softmax state over cached rows [k0, k1): Q [B, H*D]; C [B, cache_len_max, d_c];
+    lse float32 [B, H] and ctx float32 [B, H, d_c] outputs (see include/gmla.h)."""
+    for n, t in (("Q", Q), ("C", C), ("W_k", W_k)):
+        _bf16(t, n)
+    for n, t in (("lse", lse), ("ctx", ctx)):
+        if t.dtype != torch.float32:
+            raise TypeError(f"{n} must be float32")
+    B, d = Q.shape
+    H = int(num_heads)
+    D = d // H
+    _, Lmax, d_c = C.shape
+    wp, wb = _ws(workspace)
+    code = lib.gmla_attend_decode_partial(_ptr(Q), _ptr(C), B, Lmax, int(k0), int(k1), H, D, d_c, _ptr(W_k),
+                                          float(scale), _ptr(lse), _ptr(ctx), wp, wb, _stream(stream))
+    return _check(code, "gmla_attend_decode_partial") if check else code
+
+
+def gmla_decode_combine(lse, ctx, W_v, O, G=None, stream=None, check=True):
+    """Merge stacked decode states lse [n, B, H], ctx [n, B, H, d_c] (float32) into
+    O [B, H*D] = gate(W_v^(h) c^) (see include/gmla.h)."""
+    for n, t in (("W_v", W_v), ("O", O), ("G", G)):
+        _bf16(t, n)
+    for n, t in (("lse", lse), ("ctx", ctx)):
+        if t.dtype != torch.float32:
+            raise TypeError(f"{n} must be float32")
+    n_parts, B, H, d_c = ctx.shape
+    D = O.shape[-1] // H
+    code = lib.gmla_decode_combine(_ptr(lse), _ptr(ctx), n_parts, B, H, D, d_c, _ptr(W_v), _ptr(G), _ptr(O),
+                                   _stream(stream))
+    return _check(code, "gmla_decode_combine") if check else code
+
+
 def gmla_gate_out_workspace_size(M, d_model) -> int:
     return lib.gmla_gate_out_workspace_size(M, d_model)
 
 
 def gmla_gate_out(O, W_o, Y, G=None, workspace=None, stream=None, check=True):
-    """O, Y [M, d_model] (any leading shape flattened); W_o [d_model, d_model]."""
+    """Y = (sigmoid(G) (.) O) W_o^T; O, G, Y [M, d_model] (any leading shape flattened);
+    W_o [d_model, d_model]; a workspace is needed only with G."""
     for n, t in (("O", O), ("W_o", W_o), ("Y", Y), ("G", G)):
         _bf16(t, n)
     d = O.shape[-1]
@@ -314,3 +378,17 @@ def gmla_gate_out(O, W_o, Y, G=None, workspace=None, stream=None, check=True):
     wp, wb = _ws(workspace)
     code = lib.gmla_gate_out(_ptr(O), _ptr(G), _ptr(W_o), M, d, _ptr(Y), wp, wb, _stream(stream))
     return _check(code, "gmla_gate_out") if check else code
+
+
+def gmla_gate_out_heads(O, W_o, Y, head_begin, head_end, G=None, workspace=None, stream=None, check=True):
+    """Share of heads [head_begin, head_end) in Y: O, G [M, 128*(head_end-head_begin)];
+    W_o the full [d_model, d_model]; Y [M, d_model]."""
+    for n, t in (("O", O), ("W_o", W_o), ("Y", Y), ("G", G)):
+        _bf16(t, n)
+    w = O.shape[-1]
+    M = O.numel() // w
+    d = W_o.shape[0]
+    wp, wb = _ws(workspace)
+    code = lib.gmla_gate_out_heads(_ptr(O), _ptr(G), _ptr(W_o), M, d, int(head_begin), int(head_end), _ptr(Y), wp,
+                                   wb, _stream(stream))
+    return _check(code, "gmla_gate_out_heads") if check else code

@@ -1,6 +1,6 @@
 """Build libgmla.so (all CUDA sources under csrc/) for sm_100a, in-tree.
 
-    python -m causal_head_latent_b200.build [--force]
+    python causal_head_latent_b200/build.py [--force]
 
 Objects go to causal_head_latent_b200/_build/, the library to
 causal_head_latent_b200/libgmla.so.  nvcc cross-compiles without a GPU.

@@ -10,110 +10,164 @@
 //   stream   tensor-core split-KV pass over the latents (attn_latent_tc.cu):
 //            per split the running max m, sum l and acc[h,:] = sum_s p_s c_s
 //   combine  exact log-sum-exp merge of the splits, c^ = acc / l, then
-//            o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store.
+//            o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store -- or, for
+//            the partial form over a key range, the merged state itself
+//            (c^ and its log-sum-exp), which gmla_decode_combine later merges
+//            with the states of other key ranges.
+#include <math.h>
+
 #include <mutex>
 #include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "ws_layout.h"
 
 namespace gmla {
 
 int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
-                     int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l, float *part_acc,
-                     float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens, unsigned *status,
-                     cudaStream_t stream);
+                     int k_base, int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l,
+                     float *part_acc, float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens,
+                     unsigned *status, cudaStream_t stream);
 int latent_tc_tile_keys();
 
 namespace latent {
 
 constexpr int HD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
-// ---------------------------------------------------------------- absorb
-// grid (H, ceil(d_c / 128)), 128 threads: thread j owns latent column c = 128*y + j.
-__global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ Wk,
-                                                     int B, int H, int dc, float sl2, uint16_t *__restrict__ qt) {
-  extern __shared__ float qs[];  // [B][HD]
-  const int h = blockIdx.x;
-  const int c = blockIdx.y * 128 + threadIdx.x;
-  for (int i = threadIdx.x; i < B * HD; i += 128) {
-    const int b = i / HD, d = i % HD;
-    qs[i] = bf16_to_f32(Q[(size_t)b * H * HD + (size_t)h * HD + d]);
-  }
-  __syncthreads();
-  if (c >= dc) return;
-  for (int b0 = 0; b0 < B; b0 += 32) {
-    const int nb = min(32, B - b0);
-    float acc[32];
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-    // four rows d of W_k per step, so q is read from shared memory as one
-    // 16-byte broadcast per sequence instead of four
-#pragma unroll 1
-    for (int d = 0; d < HD; d += 4) {
-      float w[4];
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) w[e] = bf16_to_f32(Wk[((size_t)h * HD + d + e) * dc + c]);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j < nb) {
-          const float4 q4 = *reinterpret_cast<const float4 *>(qs + (b0 + j) * HD + d);
-          acc[j] = fmaf(q4.x, w[0], acc[j]);
-          acc[j] = fmaf(q4.y, w[1], acc[j]);
-          acc[j] = fmaf(q4.z, w[2], acc[j]);
-          acc[j] = fmaf(q4.w, w[3], acc[j]);
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < nb) qt[((size_t)(b0 + j) * H + h) * dc + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j] * sl2));
-  }
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
-// ---------------------------------------------------------------- combine + W_v + gate
-// grid (H, ceil(B / CB)), 128 threads (one per output channel of the head).
+// ---------------------------------------------------------------- absorb
+// grid (H, ceil(d_c / 128), ceil(B / AB)), 128 threads: thread j owns latent
+// column c = 128*y + j for the AB sequences b0 .. b0+AB-1.  The CTA first
+// copies its 128 x 128 tile of W_k^(h) and the AB query rows of head h into
+// shared memory with 16-byte loads that are all in flight at once, then
+// forms the products from shared memory.
+constexpr int AB = 32;
+constexpr size_t kAbsorbSmem = AB * HD * sizeof(float) + HD * 128 * sizeof(uint16_t);  // 48 KB
+
+__global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ Wk,
+                                                     int B, int H, int dc, float sl2, uint16_t *__restrict__ qt) {
+  extern __shared__ __align__(16) uint8_t absorb_sm[];
+  float *qs = reinterpret_cast<float *>(absorb_sm);                      // [AB][HD]
+  uint16_t *ws = reinterpret_cast<uint16_t *>(absorb_sm + AB * HD * 4);  // [HD][128]
+  const int h = blockIdx.x, c0 = blockIdx.y * 128, b0 = blockIdx.z * AB;
+  const int nb = min(AB, B - b0);
+  const int ncol = min(128, dc - c0);  // 64 or 128 (d_c is a multiple of 64)
+  for (int i = threadIdx.x; i < HD * 16; i += 128) {
+    const int d = i >> 4, v = i & 15;
+    if (8 * v < ncol)
+      *reinterpret_cast<uint4 *>(ws + d * 128 + 8 * v) =
+          *reinterpret_cast<const uint4 *>(Wk + ((size_t)h * HD + d) * dc + c0 + 8 * v);
+  }
+  for (int i = threadIdx.x; i < nb * 16; i += 128) {
+    const int j = i >> 4, v = i & 15;
+    const uint4 u = *reinterpret_cast<const uint4 *>(Q + (size_t)(b0 + j) * H * HD + (size_t)h * HD + 8 * v);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float *dst = qs + j * HD + 8 * v;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      dst[2 * e] = __uint_as_float(w[e] << 16);
+      dst[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  }
+  __syncthreads();
+  const int c = threadIdx.x;
+  if (c >= ncol) return;
+  float acc[AB];
+#pragma unroll
+  for (int j = 0; j < AB; ++j) acc[j] = 0.f;
+#pragma unroll 2
+  for (int d = 0; d < HD; d += 4) {
+    float w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[e] = bf16_to_f32(ws[(d + e) * 128 + c]);
+#pragma unroll
+    for (int j = 0; j < AB; ++j) {
+      if (j < nb) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(qs + j * HD + d);
+        acc[j] = fmaf(q4.x, w[0], acc[j]);
+        acc[j] = fmaf(q4.y, w[1], acc[j]);
+        acc[j] = fmaf(q4.z, w[2], acc[j]);
+        acc[j] = fmaf(q4.w, w[3], acc[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < AB; ++j)
+    if (j < nb) qt[((size_t)(b0 + j) * H + h) * dc + c0 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j] * sl2));
+}
+
+// ---------------------------------------------------------------- combine
+// grid (H, ceil(B / CB)), CT threads.  Phase 1: warp bb computes the weights
+// 2^(m_s - M) / sum_s l_s 2^(m_s - M) of the S partial states of sequence
+// b0 + bb (lanes over s).  Phase 2: c^ = sum_s w_s acc_s over all (sequence,
+// column) pairs, 16-byte loads with eight states in flight per thread.
+// Phase 3 (full form): o_h = W_v^(h) c^, two threads per output row (one half
+// of d_c each), then the gate and the bfloat16 store.  The partial form
+// stores c^ and the merged log-sum-exp instead.
 constexpr int CB = 8;
+constexpr int CT = 256;
+static_assert(CT / 32 == CB, "one warp per sequence in phase 1");
 
 struct CombineParams {
-  const float *part_m, *part_l, *part_acc;
+  const float *part_m, *part_l, *part_acc;  // [S,B,H] (m scaled by m_scale to log2 units), [S,B,H] or null (= 1),
+                                            // [S,B,H,dc]
+  float m_scale;
   int n_splits, B, H, dc;
   const uint16_t *Wv, *G;
   uint16_t *O;
-  float *lse2;  // [B,H] log2-domain log-sum-exp (for the debug weights)
+  float *lse2;                   // full form: [B,H] log2-domain log-sum-exp (for the debug weights), may be null
+  float *out_lse, *out_chat;     // partial form: [B,H] natural-log log-sum-exp, [B,H,dc] c^
 };
 
-// grid (H, ceil(B / CB)), CT threads.  Per-split weights exp2(m_s - M) / L are
-// computed once per sequence; the merge runs over all (sequence, column) pairs;
-// two threads share one output row of W_v^(h) (one half of d_c each).
-constexpr int CT = 256;
-
+template <bool kPartial>
 __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
-  extern __shared__ float sm[];  // chat [CB][dc] | split weights [CB][n_splits]
+  extern __shared__ __align__(16) float csm[];  // chat [CB][dc] | split weights [CB][n_splits]
   const int h = blockIdx.x, b0 = blockIdx.y * CB;
   const int nb = min(CB, P.B - b0);
   const int dc = P.dc, S = P.n_splits;
-  float *chat = sm;
-  float *wsp = sm + CB * dc;
-  if (threadIdx.x < nb) {
-    const int b = b0 + threadIdx.x;
+  float *chat = csm;
+  float *wsp = csm + CB * dc;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < nb) {
+    const int b = b0 + warp;
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, P.part_m[((size_t)s * P.B + b) * P.H + h]);
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, P.part_m[((size_t)s * P.B + b) * P.H + h] * P.m_scale);
+    M = warp_max(M);
     float Lsum = 0.f;
-    for (int s = 0; s < S; ++s) {
+    for (int s = lane; s < S; s += 32) {
       const size_t i = ((size_t)s * P.B + b) * P.H + h;
-      const float e = (P.part_m[i] == -INFINITY) ? 0.f : fast_exp2(P.part_m[i] - M);
-      wsp[threadIdx.x * S + s] = e;
-      Lsum += P.part_l[i] * e;
+      const float m = P.part_m[i] * P.m_scale;
+      const float e = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
+      wsp[warp * S + s] = e;
+      Lsum += (P.part_l ? P.part_l[i] : 1.f) * e;
     }
-    const float inv = 1.f / Lsum;
-    for (int s = 0; s < S; ++s) wsp[threadIdx.x * S + s] *= inv;
-    if (P.lse2) P.lse2[(size_t)b * P.H + h] = M + __log2f(Lsum);
+    Lsum = warp_sum(Lsum);
+    // no visible key in any state: every weight 0, c^ = 0, log-sum-exp -inf
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    __syncwarp();
+    for (int s = lane; s < S; s += 32) wsp[warp * S + s] *= inv;
+    if (lane == 0) {
+      const float l2 = Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY;
+      if (kPartial)
+        P.out_lse[(size_t)b * P.H + h] = l2 * kLn2;
+      else if (P.lse2)
+        P.lse2[(size_t)b * P.H + h] = l2;
+    }
   }
   __syncthreads();
-  // c^ = sum_s w_s acc_s: four latent columns per thread (16-byte loads) and
-  // eight splits' loads in flight before their multiply-adds.
   {
     const size_t split_stride4 = (size_t)P.B * P.H * dc / 4;
     for (int i4 = threadIdx.x; i4 < nb * dc / 4; i4 += CT) {
@@ -125,7 +179,7 @@ __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
         float4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          // an empty split (weight 0) left no acc: never read it
+          // an empty state (weight 0) left no acc: never read it
           v[u] = (s0 + u < S && w[s0 + u] != 0.f) ? src[(size_t)(s0 + u) * split_stride4]
                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -138,9 +192,13 @@ __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
           a.w = fmaf(ws, v[u].w, a.w);
         }
       }
-      *reinterpret_cast<float4 *>(chat + bb * dc + c) = a;
+      if (kPartial)
+        *reinterpret_cast<float4 *>(P.out_chat + ((size_t)(b0 + bb) * P.H + h) * dc + c) = a;
+      else
+        *reinterpret_cast<float4 *>(chat + bb * dc + c) = a;
     }
   }
+  if (kPartial) return;
   __syncthreads();
   const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
   const int c_lo = half * (dc / 2), c_hi = c_lo + dc / 2;
@@ -195,79 +253,55 @@ __global__ void weights_fix_varlen_kernel(float *w, const float *lse2, const int
   }
 }
 
+// The state of an empty key range: log-sum-exp -inf, c^ = 0.
+__global__ void empty_state_kernel(float *lse, float *chat, size_t n_lse, size_t n_chat) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_chat; i += (size_t)gridDim.x * blockDim.x) {
+    chat[i] = 0.f;
+    if (i < n_lse) lse[i] = -INFINITY;
+  }
+}
+
 }  // namespace latent
 
 // ------------------------------------------------------------------ split planning and workspace
 
-static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-// Split count for B sequences of L keys: fill whole waves of the 148 SMs of a
-// B200 (one CTA per SM) while keeping the float32 partial states small next to
-// the cache.  A pure function of (B, L) so the workspace size never depends on
-// the device.
 void latent_plan(long long B, long long L, int *n_splits, int *keys_per_split) {
-  const int KT = latent_tc_tile_keys();
-  const long long tiles = (L + KT - 1) / KT;
-  double best = 1e30;
-  long long best_s = 1;
-  for (long long s = 1; s <= 64 && s <= tiles; ++s) {
-    const long long ctas = B * s;
-    const long long waves = (ctas + 147) / 148;
-    const double eff = (double)ctas / (double)(waves * 148);
-    const double overhead = (double)s * 96 * 512 * 8 / ((double)L * 512 * 2 + 1.0);
-    const double cost = 1.0 / eff + overhead;
-    if (cost < best - 1e-9) {
-      best = cost;
-      best_s = s;
-    }
-  }
-  long long kps = ((tiles + best_s - 1) / best_s) * KT;
-  long long s = (L + kps - 1) / kps;  // no empty split
-  *n_splits = (int)s;
-  *keys_per_split = (int)kps;
-}
-
-// Workspace layout (each region 256-byte aligned):
-//   q~ bf16 [B,H,dc] | m, l float [S,B,H] each | acc float [S,B,H,dc] | lse2 float [B,H]
-static size_t latent_workspace_bytes_for(long long B, long long H, long long dc, long long S) {
-  return align256(2 * B * H * dc) + 2 * align256(sizeof(float) * S * B * H) + align256(sizeof(float) * S * B * H * dc) +
-         align256(sizeof(float) * B * H);
+  latent_plan(B, L, latent_tc_tile_keys(), n_splits, keys_per_split);
 }
 
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc) {
   int S, kps;
   latent_plan(B, L, &S, &kps);
-  return latent_workspace_bytes_for(B, H, dc, S);
+  return latent_layout_bytes(B, H, dc, S, false);
 }
 
 // With per-sequence lengths the plan follows cache_len_max, and the workspace
 // also holds one 128-byte tensor map and one int32 length per sequence.
 size_t latent_varlen_workspace_bytes(long long B, long long cache_len_max, long long H, long long dc) {
-  return latent_workspace_bytes(B, cache_len_max, H, dc) + align256((size_t)B * sizeof(CUtensorMap)) +
-         align256((size_t)B * sizeof(int));
+  int S, kps;
+  latent_plan(B, cache_len_max, &S, &kps);
+  return latent_layout_bytes(B, H, dc, S, true);
 }
 
-// The three launches for a given split plan (S splits of kps keys) and workspace.
+// The three launches for a given split plan (S splits of kps keys over the
+// key range [a.k0, a.L), or [0, lens[b]) per sequence) and workspace.
 static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaStream_t stream) {
   using namespace latent;
-  uint8_t *ws = static_cast<uint8_t *>(a.workspace);
-  uint16_t *qt = reinterpret_cast<uint16_t *>(ws);
-  ws += align256(2 * (size_t)a.B * a.H * a.dc);
-  float *pm = reinterpret_cast<float *>(ws);
-  ws += align256(sizeof(float) * (size_t)S * a.B * a.H);
-  float *pl = reinterpret_cast<float *>(ws);
-  ws += align256(sizeof(float) * (size_t)S * a.B * a.H);
-  float *pacc = reinterpret_cast<float *>(ws);
-  ws += align256(sizeof(float) * (size_t)S * a.B * a.H * a.dc);
-  float *lse2 = reinterpret_cast<float *>(ws);
-  ws += align256(sizeof(float) * (size_t)a.B * a.H);
+  static_assert(sizeof(CUtensorMap) == kTensorMapBytes, "tensor map size");
+  uint8_t *base = static_cast<uint8_t *>(a.workspace);
+  const LatentLayout lay = latent_layout(reinterpret_cast<uintptr_t>(base), a.B, a.H, a.dc, S, a.lens != nullptr);
+  uint16_t *qt = reinterpret_cast<uint16_t *>(base + lay.qt);
+  float *pm = reinterpret_cast<float *>(base + lay.pm);
+  float *pl = reinterpret_cast<float *>(base + lay.pl);
+  float *pacc = reinterpret_cast<float *>(base + lay.pacc);
+  float *lse2 = reinterpret_cast<float *>(base + lay.lse2);
   CUtensorMap *maps = nullptr;
   int *lens_dev = nullptr;
   if (a.lens) {
-    // per-sequence 2-D latent maps (d_c, lens[b]) and lengths, copied before the launches
-    maps = reinterpret_cast<CUtensorMap *>(ws);
-    ws += align256((size_t)a.B * sizeof(CUtensorMap));
-    lens_dev = reinterpret_cast<int *>(ws);
+    // per-sequence 2-D latent maps (d_c, lens[b]) and lengths, copied before the launches;
+    // the map region starts on a 256-byte boundary (TMA reads maps at 64-byte alignment)
+    maps = reinterpret_cast<CUtensorMap *>(base + lay.maps);
+    lens_dev = reinterpret_cast<int *>(base + lay.lens);
     std::vector<CUtensorMap> hm((size_t)a.B);
     std::vector<int> hl((size_t)a.B);
     for (int b = 0; b < a.B; ++b) {
@@ -283,27 +317,22 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
       return -1;
   }
 
-  {
-    const size_t shm = sizeof(float) * a.B * HD;
-    if (shm > 48 * 1024 &&
-        cudaFuncSetAttribute(absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm) != cudaSuccess)
-      return -1;
-    absorb_kernel<<<dim3(a.H, (a.dc + 127) / 128), 128, shm, stream>>>(a.Q, a.Wk, a.B, a.H, a.dc,
-                                                                      a.scale * kLog2e, qt);
-  }
+  absorb_kernel<<<dim3(a.H, (a.dc + 127) / 128, (a.B + AB - 1) / AB), 128, kAbsorbSmem, stream>>>(
+      a.Q, a.Wk, a.B, a.H, a.dc, a.scale * kLog2e, qt);
   {
     CUtensorMap tq, tc;
     const long long dq[3] = {a.dc, a.H, a.B}, sq[2] = {a.dc, (long long)a.H * a.dc};
     const unsigned bq[3] = {64, 96, 1};
     if (!make_tmap_bf16(&tq, qt, 3, dq, sq, bq)) return -1;
-    // The key extent is L, not cache_len_max: rows of a ragged last tile past
-    // L read as zeros, never as whatever the unwritten cache rows hold.
+    // The key extent is L (the end of the key range), not cache_len_max: rows of
+    // a ragged last tile past L read as zeros, never as whatever the unwritten
+    // cache rows hold.
     const long long dcm[3] = {a.dc, a.L, a.B}, scm[2] = {a.dc, a.cache_len_max * a.dc};
     const unsigned bc[3] = {64, (unsigned)latent_tc_tile_keys(), 1};
     if (!make_tmap_bf16(&tc, a.C, 3, dcm, scm, bc)) return -1;
     const int w_ld = a.lens ? (int)a.cache_len_max : a.L;
-    if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, a.H, a.dc, S, kps, pm, pl, pacc, a.weights, w_ld, maps,
-                         lens_dev, a.status, stream) != 0)
+    if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, (int)a.k0, a.H, a.dc, S, kps, pm, pl, pacc,
+                         a.weights, w_ld, maps, lens_dev, a.status, stream) != 0)
       return -1;
   }
   {
@@ -311,6 +340,7 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     P.part_m = pm;
     P.part_l = pl;
     P.part_acc = pacc;
+    P.m_scale = 1.f;
     P.n_splits = S;
     P.B = a.B;
     P.H = a.H;
@@ -319,7 +349,14 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     P.G = a.G;
     P.O = a.O;
     P.lse2 = lse2;
-    combine_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), CT, sizeof(float) * (CB * a.dc + CB * S), stream>>>(P);
+    P.out_lse = a.out_lse;
+    P.out_chat = a.out_chat;
+    const dim3 grid(a.H, (a.B + CB - 1) / CB);
+    const size_t shm = sizeof(float) * (CB * a.dc + CB * S);
+    if (a.out_chat)
+      combine_kernel<true><<<grid, CT, shm, stream>>>(P);
+    else
+      combine_kernel<false><<<grid, CT, shm, stream>>>(P);
   }
   if (a.weights && a.lens)
     weights_fix_varlen_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, lens_dev, a.H, a.B * a.H,
@@ -331,8 +368,37 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
 
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream) {
   int S, kps;
-  latent_plan(a.B, a.lens ? a.cache_len_max : a.L, &S, &kps);
+  latent_plan(a.B, a.lens ? a.cache_len_max : a.L - a.k0, &S, &kps);
   return launch_attend_latent_plan(a, S, kps, stream);
+}
+
+int launch_latent_empty_state(float *lse, float *chat, long long B, long long H, long long dc, cudaStream_t stream) {
+  latent::empty_state_kernel<<<2 * num_sms(), 256, 0, stream>>>(lse, chat, (size_t)(B * H), (size_t)(B * H * dc));
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// Merge n partial states (natural-log lse [n,B,H], c^ [n,B,H,dc]), apply
+// W_v^(h) and the gate.
+int launch_latent_combine(const float *lse, const float *chat, int n, int B, int H, int dc, const uint16_t *Wv,
+                          const uint16_t *G, uint16_t *O, cudaStream_t stream) {
+  using namespace latent;
+  CombineParams P;
+  P.part_m = lse;
+  P.part_l = nullptr;
+  P.part_acc = chat;
+  P.m_scale = kLog2e;
+  P.n_splits = n;
+  P.B = B;
+  P.H = H;
+  P.dc = dc;
+  P.Wv = Wv;
+  P.G = G;
+  P.O = O;
+  P.lse2 = nullptr;
+  P.out_lse = nullptr;
+  P.out_chat = nullptr;
+  combine_kernel<false><<<dim3(H, (B + CB - 1) / CB), CT, sizeof(float) * (CB * dc + CB * n), stream>>>(P);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 // ------------------------------------------------------------------ decode without a caller workspace
@@ -360,8 +426,11 @@ static std::mutex g_decode_scratch_mu;
 
 // Device address of the scratch array on the current device.  The symbol's
 // name is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
-static void *decode_scratch_address() {
+// device (with that device current) and cached.  The lookup also loads this
+// file's device code on that device, which commits the array's memory; the
+// per-device set-up of every entry point calls this, so the first call of
+// any entry point on a device is the one that commits it.
+void *latent_noalloc_scratch_address() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(g_decode_scratch_mu);
@@ -380,14 +449,16 @@ size_t latent_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 int launch_attend_latent_noalloc(const LatentArgs &args, cudaStream_t stream) {
   int S, kps;
   latent_plan(args.B, args.L, &S, &kps);
-  // fewer splits when the default plan's partial states do not fit
-  while (S > 1 && latent_workspace_bytes_for(args.B, args.H, args.dc, S) > kNoAllocScratchBytes) --S;
-  if (latent_workspace_bytes_for(args.B, args.H, args.dc, S) > kNoAllocScratchBytes) return -3;
+  // fewer splits when the default plan's partial states do not fit (the array
+  // is 256-byte aligned, so the layout starts at its first byte)
+  auto fits = [&](int s) { return latent_layout(0, args.B, args.H, args.dc, s, false).end <= kNoAllocScratchBytes; };
+  while (S > 1 && !fits(S)) --S;
+  if (!fits(S)) return -3;
   const int KT = latent_tc_tile_keys();
   const long long tiles = (args.L + KT - 1) / KT;
   kps = (int)(((tiles + S - 1) / S) * KT);
   S = (int)((args.L + kps - 1) / kps);  // no empty split
-  void *scratch = decode_scratch_address();
+  void *scratch = latent_noalloc_scratch_address();
   if (!scratch) return -1;
   LatentArgs a = args;
   a.workspace = scratch;

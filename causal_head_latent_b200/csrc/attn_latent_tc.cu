@@ -98,6 +98,7 @@ struct Params {
   const uint16_t *C;  // latent cache [B, Lmax, dc] (for the L2 prefetch stream)
   long long Lmax;
   int B, L, H, dc, n_splits, keys_per_split;
+  int k_base;                         // first key of split 0 (the keys of a sequence are [k_base, L))
   float *part_m, *part_l, *part_acc;  // [S,B,H], [S,B,H], [S,B,H,512]
   float *weights;                     // optional raw log2-domain scores [B,H,w_ld]
   int w_ld;                           // row stride of weights (L, or Lmax with per-sequence lengths)
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int b = blockIdx.x / p.n_splits;
   const int split = blockIdx.x % p.n_splits;
   const int Lb = p.lens ? p.lens[b] : p.L;
-  const int k_begin = split * p.keys_per_split;
+  const int k_begin = p.k_base + split * p.keys_per_split;
   const int k_end = min(Lb, k_begin + p.keys_per_split);
   if (k_end <= k_begin) {
     // A split past the end of a shorter sequence: an empty partial state,
@@ -462,9 +463,9 @@ size_t smem_bytes() {
 int latent_tc_tile_keys() { return latent_tc::KT; }
 
 int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
-                     int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l, float *part_acc,
-                     float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens, unsigned *status,
-                     cudaStream_t stream) {
+                     int k_base, int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l,
+                     float *part_acc, float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens,
+                     unsigned *status, cudaStream_t stream) {
   using namespace latent_tc;
   auto kern = latent_decode_kernel;
   const size_t smem = smem_bytes();
@@ -474,6 +475,7 @@ int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint
   p.Lmax = Lmax;
   p.B = B;
   p.L = L;
+  p.k_base = k_base;
   p.H = H;
   p.dc = dc;
   p.n_splits = n_splits;

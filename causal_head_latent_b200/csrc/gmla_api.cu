@@ -13,6 +13,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "ws_layout.h"
 
 namespace gmla {
 
@@ -40,6 +41,11 @@ static bool device_setup(int dev) {
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
   g_num_sms[dev] = sms;
   g_status_ptr[dev] = static_cast<unsigned *>(p);
+  // Commit the scratch array of gmla_attend_decode_noalloc on this device now
+  // (its lookup loads the device code that holds it), so that a caller's first
+  // call of any entry point, not its first no-alloc decode, is the one that
+  // takes that memory.  A failure here is reported by the no-alloc call itself.
+  (void)latent_noalloc_scratch_address();
   return true;
 }
 
@@ -161,17 +167,14 @@ gmla_status gmla_selftest_wait_timeout(unsigned milliseconds, gmla_stream_t stre
 
 // ------------------------------------------------------------------ projections
 
-size_t gmla_latent_project_workspace_size(int64_t B, int64_t T, int64_t d_model, int64_t d_c) {
-  (void)B; (void)T; (void)d_model; (void)d_c;
-  return 0;
-}
-
-gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model, const gmla_bf16 *W_q,
-                                const gmla_bf16 *W_g, const gmla_bf16 *W_c, int64_t d_c, const gmla_bf16 *W_k,
-                                const gmla_bf16 *W_v, gmla_bf16 *Q, gmla_bf16 *G, gmla_bf16 *C,
-                                int64_t cache_len_max, int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V,
-                                void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
-  (void)workspace; (void)workspace_bytes;
+// [Q | G | C] = X [W_q; W_g; W_c]^T and [K | V] = C [W_k; W_v]^T for the heads
+// [h0, h1) (rows 128*h0 .. 128*h1-1 of W_q, W_g, W_k, W_v; the latent is
+// always full width).
+static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model, int64_t h0,
+                                        int64_t h1, const gmla_bf16 *W_q, const gmla_bf16 *W_g, const gmla_bf16 *W_c,
+                                        int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v, gmla_bf16 *Q,
+                                        gmla_bf16 *G, gmla_bf16 *C, int64_t cache_len_max, int64_t cache_pos,
+                                        gmla_bf16 *K, gmla_bf16 *V, gmla_stream_t stream) {
   if (!X || B <= 0 || T <= 0 || d_model <= 0 || d_c <= 0) return GMLA_ERR_ARG;
   if ((Q && !W_q) || (G && !W_g) || (C && !W_c) || (K && !W_k) || (V && !W_v)) return GMLA_ERR_ARG;
   if ((K || V) && !C) return GMLA_ERR_ARG;
@@ -180,11 +183,13 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return GMLA_ERR_ARG;
   if (d_model % 128 != 0 || d_c % 64 != 0) return GMLA_ERR_UNSUPPORTED;
+  if (h0 < 0 || h1 <= h0 || h1 > d_model / 128) return GMLA_ERR_ARG;
   if (B * T > 0x7fffffffLL || cache_len_max > 0x7fffffffLL || B > 65535) return GMLA_ERR_UNSUPPORTED;
   unsigned *st = status_ptr();
   if (!st) return GMLA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long M = B * T;
+  const long long w = 128 * (h1 - h0);  // output width of Q, G, K, V
 
   // [Q | G | C] = X [W_q; W_g; W_c]^T
   {
@@ -199,11 +204,12 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
     ga.K = (int)d_model;
     ga.status = st;
     int np = 0;
-    const gmla_bf16 *Ws[3] = {W_q, W_g, W_c};
+    const gmla_bf16 *Ws[3] = {W_q ? W_q + 128 * h0 * d_model : nullptr, W_g ? W_g + 128 * h0 * d_model : nullptr,
+                              W_c};
     gmla_bf16 *Os[3] = {Q, G, C};
     for (int i = 0; i < 3; ++i) {
       if (!Os[i]) continue;
-      const long long N = i == 2 ? d_c : d_model;
+      const long long N = i == 2 ? d_c : w;
       const long long dB[2] = {d_model, N}, sB[1] = {d_model};
       const unsigned bB[2] = {64, 256};
       if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
@@ -218,7 +224,7 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
       } else {
         o.rows_per_b = M;
         o.sb = 0;
-        o.st = d_model;
+        o.st = w;
         o.off = 0;
       }
       ++np;
@@ -239,19 +245,19 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
     ga.K = (int)d_c;
     ga.status = st;
     int np = 0;
-    const gmla_bf16 *Ws[2] = {W_k, W_v};
+    const gmla_bf16 *Ws[2] = {W_k ? W_k + 128 * h0 * d_c : nullptr, W_v ? W_v + 128 * h0 * d_c : nullptr};
     gmla_bf16 *Os[2] = {K, V};
     for (int i = 0; i < 2; ++i) {
       if (!Os[i]) continue;
-      const long long dB[2] = {d_c, d_model}, sB[1] = {d_c};
+      const long long dB[2] = {d_c, w}, sB[1] = {d_c};
       const unsigned bB[2] = {64, 256};
       if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
       GemmOut &o = ga.prob[np];
       o.out = Os[i];
-      o.N = (int)d_model;
+      o.N = (int)w;
       o.rows_per_b = M;
       o.sb = 0;
-      o.st = d_model;
+      o.st = w;
       o.off = 0;
       ++np;
     }
@@ -259,6 +265,26 @@ gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_
     if (launch_gemm(tmA, tmB, ga, s) != 0) return GMLA_ERR_CUDA;
   }
   return GMLA_OK;
+}
+
+gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model, const gmla_bf16 *W_q,
+                                const gmla_bf16 *W_g, const gmla_bf16 *W_c, int64_t d_c, const gmla_bf16 *W_k,
+                                const gmla_bf16 *W_v, gmla_bf16 *Q, gmla_bf16 *G, gmla_bf16 *C,
+                                int64_t cache_len_max, int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V,
+                                gmla_stream_t stream) {
+  if (d_model <= 0) return GMLA_ERR_ARG;
+  if (d_model % 128 != 0) return GMLA_ERR_UNSUPPORTED;
+  return latent_project_heads(X, B, T, d_model, 0, d_model / 128, W_q, W_g, W_c, d_c, W_k, W_v, Q, G, C,
+                              cache_len_max, cache_pos, K, V, stream);
+}
+
+gmla_status gmla_latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model, int64_t head_begin,
+                                      int64_t head_end, const gmla_bf16 *W_q, const gmla_bf16 *W_g,
+                                      const gmla_bf16 *W_c, int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v,
+                                      gmla_bf16 *Q, gmla_bf16 *G, gmla_bf16 *C, int64_t cache_len_max,
+                                      int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V, gmla_stream_t stream) {
+  return latent_project_heads(X, B, T, d_model, head_begin, head_end, W_q, W_g, W_c, d_c, W_k, W_v, Q, G, C,
+                              cache_len_max, cache_pos, K, V, stream);
 }
 
 // ------------------------------------------------------------------ K/V expansion of cached latents
@@ -370,7 +396,7 @@ gmla_status gmla_attend_prefill(const gmla_bf16 *Q, const int64_t q_strides[3], 
 
 size_t gmla_attend_prefill_varlen_workspace_size(int64_t B) {
   if (B <= 0) return 0;
-  return 3 * (size_t)B * sizeof(CUtensorMap) + 2 * (size_t)B * sizeof(int) + 256;
+  return prefill_varlen_layout_bytes(B);
 }
 
 gmla_status gmla_attend_prefill_varlen(const gmla_bf16 *Q, const int64_t q_strides[3], const gmla_bf16 *K,
@@ -401,9 +427,11 @@ gmla_status gmla_attend_prefill_varlen(const gmla_bf16 *Q, const int64_t q_strid
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   // per-sequence 3-D maps (D, length, H) and lengths, copied into the workspace
-  uint8_t *ws = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(workspace) + 127) & ~uintptr_t(127));
-  CUtensorMap *maps = reinterpret_cast<CUtensorMap *>(ws);
-  int *lens = reinterpret_cast<int *>(ws + 3 * (size_t)B * sizeof(CUtensorMap));
+  // (the map region starts on a 256-byte boundary: TMA reads maps at 64-byte alignment)
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const PrefillVarlenLayout lay = prefill_varlen_layout(reinterpret_cast<uintptr_t>(ws), B);
+  CUtensorMap *maps = reinterpret_cast<CUtensorMap *>(ws + lay.maps);
+  int *lens = reinterpret_cast<int *>(ws + lay.lens);
   std::vector<CUtensorMap> hm(3 * (size_t)B);
   std::vector<int> hl(2 * (size_t)B);
   const unsigned box[3] = {64, 128, 1};
@@ -507,6 +535,58 @@ gmla_status gmla_attend_decode_varlen(const gmla_bf16 *Q, const gmla_bf16 *C, in
   return launch_attend_latent(a, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ decode state over a key range, and its merge
+
+size_t gmla_attend_decode_partial_workspace_size(int64_t B, int64_t k0, int64_t k1, int64_t H, int64_t d_c) {
+  if (B <= 0 || k0 < 0 || k1 <= k0 || H <= 0 || d_c <= 0) return 0;
+  return latent_workspace_bytes(B, k1 - k0, H, d_c);
+}
+
+gmla_status gmla_attend_decode_partial(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B, int64_t cache_len_max,
+                                       int64_t k0, int64_t k1, int64_t H, int64_t D_h, int64_t d_c,
+                                       const gmla_bf16 *W_k, float scale, float *lse, float *ctx, void *workspace,
+                                       size_t workspace_bytes, gmla_stream_t stream) {
+  if (!Q || !C || !W_k || !lse || !ctx) return GMLA_ERR_ARG;
+  if (B <= 0 || H <= 0 || D_h <= 0 || d_c <= 0 || k0 < 0 || k1 < k0 || k1 > cache_len_max) return GMLA_ERR_ARG;
+  const void *ptrs[] = {Q, C, W_k, lse, ctx, workspace};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (D_h != 128 || d_c % 64 != 0 || d_c > 512 || H > 96) return GMLA_ERR_UNSUPPORTED;
+  if (B > 65535 || cache_len_max > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  if (k1 > k0 && (!workspace || workspace_bytes < latent_workspace_bytes(B, k1 - k0, H, d_c)))
+    return GMLA_ERR_WORKSPACE;
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k1 == k0) return launch_latent_empty_state(lse, ctx, B, H, d_c, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+  if (scale <= 0.f) scale = 1.0f / sqrtf((float)D_h);
+  LatentArgs a{};
+  a.Q = Q; a.C = C; a.Wk = W_k; a.Wv = nullptr; a.G = nullptr; a.O = nullptr; a.weights = nullptr;
+  a.cache_len_max = cache_len_max;
+  a.B = (int)B; a.L = (int)k1; a.H = (int)H; a.dc = (int)d_c;
+  a.scale = scale; a.workspace = workspace; a.status = st;
+  a.k0 = k0; a.out_lse = lse; a.out_chat = ctx;
+  return launch_attend_latent(a, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
+gmla_status gmla_decode_combine(const float *lse, const float *ctx, int64_t n_parts, int64_t B, int64_t H,
+                                int64_t D_h, int64_t d_c, const gmla_bf16 *W_v, const gmla_bf16 *G, gmla_bf16 *O,
+                                gmla_stream_t stream) {
+  if (!lse || !ctx || !W_v || !O) return GMLA_ERR_ARG;
+  if (n_parts <= 0 || B <= 0 || H <= 0 || D_h <= 0 || d_c <= 0) return GMLA_ERR_ARG;
+  const void *ptrs[] = {lse, ctx, W_v, G, O};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GMLA_ERR_ARG;
+  if (D_h != 128 || d_c % 64 != 0 || d_c > 512 || n_parts > 1024) return GMLA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return GMLA_ERR_UNSUPPORTED;
+  unsigned *st = status_ptr();
+  if (!st) return GMLA_ERR_CUDA;
+  return launch_latent_combine(lse, ctx, (int)n_parts, (int)B, (int)H, (int)d_c, W_v, G, O,
+                               static_cast<cudaStream_t>(stream)) == 0
+             ? GMLA_OK
+             : GMLA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ decode without a caller workspace
 
 size_t gmla_attend_decode_noalloc_max_bytes(void) { return latent_noalloc_scratch_bytes(); }
@@ -538,31 +618,45 @@ gmla_status gmla_attend_decode_noalloc(const gmla_bf16 *Q, const gmla_bf16 *C, i
 // ------------------------------------------------------------------ output projection
 
 size_t gmla_gate_out_workspace_size(int64_t M, int64_t d_model) {
-  (void)M; (void)d_model;
-  return 0;
+  if (M <= 0 || d_model <= 0) return 0;
+  return gate_out_layout_bytes(M, d_model);
 }
 
-gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M, int64_t d_model,
-                          gmla_bf16 *Y, void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
-  (void)workspace; (void)workspace_bytes;
+// Y = (sigmoid(G) (.) O) W_o[:, 128*h0 .. 128*h1)^T with O, G [M, 128*(h1-h0)].
+static gmla_status gate_out_heads(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M,
+                                  int64_t d_model, int64_t h0, int64_t h1, gmla_bf16 *Y, void *workspace,
+                                  size_t workspace_bytes, gmla_stream_t stream) {
   if (!O || !W_o || !Y || M <= 0 || d_model <= 0) return GMLA_ERR_ARG;
-  if (!aligned16(O) || !aligned16(W_o) || !aligned16(Y)) return GMLA_ERR_ARG;
-  if (G) return GMLA_ERR_UNSUPPORTED;
+  if (!aligned16(O) || !aligned16(W_o) || !aligned16(Y) || (G && !aligned16(G)) ||
+      (workspace && !aligned16(workspace)))
+    return GMLA_ERR_ARG;
   if (d_model % 128 != 0 || M > 0x7fffffffLL) return GMLA_ERR_UNSUPPORTED;
+  if (h0 < 0 || h1 <= h0 || h1 > d_model / 128) return GMLA_ERR_ARG;
+  const long long w = 128 * (h1 - h0);  // width of O and G
+  if (G && (!workspace || workspace_bytes < gate_out_layout_bytes(M, w))) return GMLA_ERR_WORKSPACE;
   unsigned *st = status_ptr();
   if (!st) return GMLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const gmla_bf16 *A = O;
+  if (G) {  // the gated context, staged in the workspace
+    gmla_bf16 *gated = reinterpret_cast<gmla_bf16 *>(static_cast<uint8_t *>(workspace) +
+                                                     gate_out_layout_offset(reinterpret_cast<uintptr_t>(workspace)));
+    if (launch_gate(O, G, gated, (size_t)M * w, s) != 0) return GMLA_ERR_CUDA;
+    A = gated;
+  }
   GemmArgs ga{};
   CUtensorMap tmA, tmB[3];
-  const long long dA[3] = {d_model, M, 1}, sA[2] = {d_model, M * d_model};
+  const long long dA[3] = {w, M, 1}, sA[2] = {w, M * w};
   const unsigned bA[3] = {64, 128, 1};
-  if (!make_tmap_bf16(&tmA, O, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
-  const long long dB[2] = {d_model, d_model}, sB[1] = {d_model};
+  if (!make_tmap_bf16(&tmA, A, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+  // columns 128*h0 .. 128*h1-1 of every row of W_o: a strided sub-matrix
+  const long long dB[2] = {w, d_model}, sB[1] = {d_model};
   const unsigned bB[2] = {64, 256};
-  if (!make_tmap_bf16(&tmB[0], W_o, 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+  if (!make_tmap_bf16(&tmB[0], W_o + 128 * h0, 2, dB, sB, bB)) return GMLA_ERR_CUDA;
   ga.a_rows = (int)M;
   ga.a_batches = 1;
   ga.a_row0 = 0;
-  ga.K = (int)d_model;
+  ga.K = (int)w;
   ga.status = st;
   ga.n_problems = 1;
   ga.prob[0].out = Y;
@@ -571,7 +665,20 @@ gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf1
   ga.prob[0].sb = 0;
   ga.prob[0].st = d_model;
   ga.prob[0].off = 0;
-  return launch_gemm(tmA, tmB, ga, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+  return launch_gemm(tmA, tmB, ga, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+}
+
+gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M, int64_t d_model,
+                          gmla_bf16 *Y, void *workspace, size_t workspace_bytes, gmla_stream_t stream) {
+  if (d_model <= 0) return GMLA_ERR_ARG;
+  if (d_model % 128 != 0) return GMLA_ERR_UNSUPPORTED;
+  return gate_out_heads(O, G, W_o, M, d_model, 0, d_model / 128, Y, workspace, workspace_bytes, stream);
+}
+
+gmla_status gmla_gate_out_heads(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M,
+                                int64_t d_model, int64_t head_begin, int64_t head_end, gmla_bf16 *Y, void *workspace,
+                                size_t workspace_bytes, gmla_stream_t stream) {
+  return gate_out_heads(O, G, W_o, M, d_model, head_begin, head_end, Y, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -78,14 +78,29 @@ struct LatentArgs {
   // Optional per-sequence lengths (host array of B values in 1..cache_len_max);
   // when set, L is ignored and the split plan and workspace follow cache_len_max.
   const long long *lens = nullptr;
+  // Partial form: keys [k0, L) only; the merged state goes to out_lse
+  // (natural log, [B,H]) and out_chat ([B,H,dc]) instead of O (out_chat
+  // non-null selects the partial form).
+  long long k0 = 0;
+  float *out_lse = nullptr, *out_chat = nullptr;
 };
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream);
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc);
 size_t latent_varlen_workspace_bytes(long long B, long long cache_len_max, long long H, long long dc);
+// The state of an empty key range (lse = -inf, chat = 0).
+int launch_latent_empty_state(float *lse, float *chat, long long B, long long H, long long dc, cudaStream_t stream);
+// Merge n partial states (lse [n,B,H] natural log, chat [n,B,H,dc]), then W_v and the gate into O.
+int launch_latent_combine(const float *lse, const float *chat, int n, int B, int H, int dc, const uint16_t *Wv,
+                          const uint16_t *G, uint16_t *O, cudaStream_t stream);
 // Same launches with the scratch in a fixed device array of this library
 // (no workspace argument).  Returns 0, -1 (CUDA error) or -3 (too large).
 int launch_attend_latent_noalloc(const LatentArgs &a, cudaStream_t stream);
 size_t latent_noalloc_scratch_bytes();
+// Device address of that array on the current device (looked up once per device).
+void *latent_noalloc_scratch_address();
+
+// out = sigmoid(G) (.) O over n bf16 elements (n a multiple of 8, 16-byte aligned pointers).
+int launch_gate(const uint16_t *O, const uint16_t *G, uint16_t *out, size_t n, cudaStream_t stream);
 
 int num_sms();
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current

@@ -20,14 +20,19 @@
  * ------------
  *  gmla_latent_project       projections [Q | G | C] = X [W_q; W_g; W_c]^T (C into
  *                            the cache rows) and optionally K, V of those rows
+ *  gmla_latent_project_heads   the same for a range of heads (head-parallel prefill)
  *  gmla_expand_kv            K, V of any range of cached latent rows
  *  gmla_attend_prefill       causal (or full) attention over explicit Q, K, V
  *  gmla_attend_prefill_varlen  the same over a padded batch with per-sequence
  *                            query / key lengths
  *  gmla_attend_decode        one new query per sequence over the latent cache
  *  gmla_attend_decode_varlen   the same with per-sequence cache lengths
+ *  gmla_attend_decode_partial  the softmax state of that query over a range of
+ *                            cached rows (context-parallel decode) ...
+ *  gmla_decode_combine       ... and the exact merge of such states into the output
  *  gmla_attend_decode_noalloc  gmla_attend_decode without a caller workspace
- *  gmla_gate_out             the output projection Y = O W_o^T
+ *  gmla_gate_out             the gate and output projection Y = (sigmoid(G) (.) O) W_o^T
+ *  gmla_gate_out_heads       its share for a range of heads (head-parallel prefill)
  *  gmla_get_device_status, gmla_selftest_wait_timeout, gmla_status_string,
  *  gmla_version, and a *_workspace_size query per call that needs scratch.
  *
@@ -101,20 +106,38 @@ typedef void *gmla_stream_t; /* a cudaStream_t */
  *          cache_pos + T <= cache_len_max.  Required when K or V is requested.
  *  K, V    [B, T, d_model] outputs, may be NULL.  They are expanded from the
  *          bfloat16 latents just written to C.
- *  workspace / workspace_bytes: scratch of at least
- *          gmla_latent_project_workspace_size(B, T, d_model, d_c) bytes
- *          (may be NULL when that size is 0).
- * Returns GMLA_ERR_ARG for null required pointers, d_model != 128*H shapes
- * that are not multiples of 128, cache_pos + T > cache_len_max, or
- * misalignment; GMLA_ERR_WORKSPACE for a short workspace.
+ * Needs no scratch memory.
+ * Returns GMLA_ERR_ARG for null required pointers, cache_pos + T >
+ * cache_len_max or misalignment; GMLA_ERR_UNSUPPORTED when d_model is not a
+ * multiple of 128 or d_c not a multiple of 64.
  */
 GMLA_API gmla_status gmla_latent_project(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model,
                                 const gmla_bf16 *W_q, const gmla_bf16 *W_g, const gmla_bf16 *W_c,
                                 int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v,
                                 gmla_bf16 *Q, gmla_bf16 *G, gmla_bf16 *C, int64_t cache_len_max,
-                                int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V, void *workspace,
-                                size_t workspace_bytes, gmla_stream_t stream);
-GMLA_API size_t gmla_latent_project_workspace_size(int64_t B, int64_t T, int64_t d_model, int64_t d_c);
+                                int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V, gmla_stream_t stream);
+
+/*
+ * gmla_latent_project_heads -- gmla_latent_project for the heads
+ * [head_begin, head_end) only: the share of one GPU when the heads of a layer
+ * are split over several GPUs.  Head h owns channels [128h, 128h + 128) of
+ * Q, G, K and V ("Gated MLA" page, "Split attention into heads"), i.e. rows
+ * 128h .. 128h+127 of W_q, W_g, W_k and W_v, so a head range needs only those
+ * rows; the latent C is shared by all heads and is computed in full.
+ *
+ *  W_q, W_g, W_c, W_k, W_v   the FULL weights, as for gmla_latent_project
+ *                            (only the rows of the range are read)
+ *  Q, G, K, V  [B, T, 128 * (head_end - head_begin)] outputs for the range
+ *  0 <= head_begin < head_end <= d_model / 128.  The other arguments, and the
+ *  errors, are those of gmla_latent_project; the full range gives its result.
+ */
+GMLA_API gmla_status gmla_latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T, int64_t d_model,
+                                              int64_t head_begin, int64_t head_end, const gmla_bf16 *W_q,
+                                              const gmla_bf16 *W_g, const gmla_bf16 *W_c, int64_t d_c,
+                                              const gmla_bf16 *W_k, const gmla_bf16 *W_v, gmla_bf16 *Q,
+                                              gmla_bf16 *G, gmla_bf16 *C, int64_t cache_len_max,
+                                              int64_t cache_pos, gmla_bf16 *K, gmla_bf16 *V,
+                                              gmla_stream_t stream);
 
 /*
  * gmla_expand_kv -- K = C W_k^T and V = C W_v^T for cached latent rows
@@ -248,8 +271,10 @@ GMLA_API size_t gmla_attend_decode_workspace_size(int64_t B, int64_t L, int64_t 
  *  weights optional float32 [B, H, cache_len_max]; columns at or past lens[b]
  *          are written as 0.
  *  workspace >= gmla_attend_decode_varlen_workspace_size(B, cache_len_max,
- *          H, d_c) bytes; it also receives one tensor map and one length per
- *          sequence (copied from the host on `stream` before the launches).
+ *          H, d_c) bytes, 16-byte aligned; it also receives one tensor map and
+ *          one length per sequence (copied from the host on `stream` before the
+ *          launches; the call places them on a 256-byte boundary inside the
+ *          workspace, which the reported size allows for).
  * Errors: GMLA_ERR_ARG for a null pointer or a length outside 1..cache_len_max,
  * the rest as gmla_attend_decode.
  */
@@ -261,6 +286,55 @@ GMLA_API gmla_status gmla_attend_decode_varlen(const gmla_bf16 *Q, const gmla_bf
                                               size_t workspace_bytes, gmla_stream_t stream);
 GMLA_API size_t gmla_attend_decode_varlen_workspace_size(int64_t B, int64_t cache_len_max, int64_t H,
                                                          int64_t d_c);
+
+/*
+ * gmla_attend_decode_partial -- the softmax state of one new query per
+ * sequence over the cached latent rows [k0, k1) only.  Softmax over keys
+ * ("Kimi K3 - Softmax over keys") restricted to a key subset, with its
+ * log-sum-exp, so that states of disjoint subsets merge exactly
+ * (gmla_decode_combine): the share of one GPU when the latent cache of a
+ * long context is split over several GPUs along its length (the
+ * "Le Transformer et l'attention" page's cost table: at 1M tokens the cache
+ * is 128 times that of 8K).  Same absorbed evaluation as gmla_attend_decode.
+ *
+ *  Q, C, B, cache_len_max, H, D_h, d_c, W_k, scale: as gmla_attend_decode.
+ *  0 <= k0 <= k1 <= cache_len_max; rows [k0, k1) of every sequence are read
+ *          (the query's own latent belongs to whichever range holds row L-1).
+ *  lse     float32 [B, H] output: natural log of sum_{s in [k0,k1)} exp(scale q_h.k_s)
+ *  ctx     float32 [B, H, d_c] output: sum_{s in [k0,k1)} a_s c_s, with a_s the
+ *          softmax weights normalised over [k0, k1) and c_s the latent rows
+ *          (so the head context over the range is W_v^(h) ctx[b,h,:]).
+ *          k0 == k1 gives lse = -inf and ctx = 0: an empty range.
+ *  workspace >= gmla_attend_decode_partial_workspace_size(B, k0, k1, H, d_c)
+ *          bytes (0 when k0 == k1; the pointer may then be NULL).
+ * Errors as gmla_attend_decode; GMLA_ERR_ARG also for a bad range.
+ */
+GMLA_API gmla_status gmla_attend_decode_partial(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B,
+                                               int64_t cache_len_max, int64_t k0, int64_t k1, int64_t H,
+                                               int64_t D_h, int64_t d_c, const gmla_bf16 *W_k, float scale,
+                                               float *lse, float *ctx, void *workspace, size_t workspace_bytes,
+                                               gmla_stream_t stream);
+GMLA_API size_t gmla_attend_decode_partial_workspace_size(int64_t B, int64_t k0, int64_t k1, int64_t H,
+                                                          int64_t d_c);
+
+/*
+ * gmla_decode_combine -- merge n_parts decode states of disjoint key ranges
+ * (gmla_attend_decode_partial) into the decode output: with m = max_i lse_i,
+ * w_i = exp(lse_i - m) / sum_j exp(lse_j - m), c^ = sum_i w_i ctx_i (the
+ * softmax over the union of the ranges, exact in real arithmetic), then
+ * o_h = W_v^(h) c^_h and, when G is given, the gate sigmoid(G) (.) o
+ * ("Gated MLA" page, "The channel-wise output gate").
+ *
+ *  lse     float32 [n_parts, B, H]; ctx float32 [n_parts, B, H, d_c]: the
+ *          states stacked along a leading axis (what an all-gather of the
+ *          per-GPU states produces); states with lse = -inf are skipped, and a
+ *          sequence whose states are all empty gets O = 0.
+ *  W_v     [H*D_h, d_c]; G optional gate logits [B, H*D_h]; O [B, H*D_h] output.
+ *  1 <= n_parts <= 1024.  Needs no scratch memory.
+ */
+GMLA_API gmla_status gmla_decode_combine(const float *lse, const float *ctx, int64_t n_parts, int64_t B,
+                                        int64_t H, int64_t D_h, int64_t d_c, const gmla_bf16 *W_v,
+                                        const gmla_bf16 *G, gmla_bf16 *O, gmla_stream_t stream);
 
 /*
  * gmla_attend_decode_noalloc -- gmla_attend_decode for callers that cannot
@@ -286,8 +360,12 @@ GMLA_API size_t gmla_attend_decode_varlen_workspace_size(int64_t B, int64_t cach
  *    rewrites all the scratch it reads, so nothing needs clearing.  Calls whose
  *    GPU work overlaps (different streams, or unordered host threads) race on
  *    the array: order them on one stream.
- *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current).
+ *  - The array's device address is looked up once per device, with that
+ *    device current, by the first call of ANY entry point of this library on
+ *    that device (gmla_get_device_status included); that lookup loads the
+ *    library's device code there and commits the 32 MiB.  A caller that
+ *    reserves all free device memory for its own pool should therefore make
+ *    one call (gmla_get_device_status suffices) before reserving it.
  */
 GMLA_API gmla_status gmla_attend_decode_noalloc(const gmla_bf16 *Q, const gmla_bf16 *C, int64_t B,
                                                int64_t cache_len_max, int64_t L, int64_t H, int64_t D_h,
@@ -297,19 +375,47 @@ GMLA_API gmla_status gmla_attend_decode_noalloc(const gmla_bf16 *Q, const gmla_b
 GMLA_API size_t gmla_attend_decode_noalloc_max_bytes(void);
 
 /*
- * gmla_gate_out -- the output projection Y = O W_o^T over M = B*T rows.
- * "Gated MLA" page, "The channel-wise output gate" (gate before W_o) and
- * step 6.  The gate is applied upstream (gmla_attend_prefill and
- * gmla_attend_decode take G); passing G != NULL here returns
- * GMLA_ERR_UNSUPPORTED.
+ * gmla_gate_out -- the gate and the output projection over M = B*T rows:
+ * Y = (sigmoid(G) (.) O) W_o^T ("Gated MLA" page, "The channel-wise output
+ * gate": the gate acts channel by channel, before W_o; step 6).  The
+ * attention calls already fuse the gate (gmla_attend_prefill and
+ * gmla_attend_decode take G), so the usual call passes their gated output
+ * with G = NULL; a caller holding an ungated context passes its gate logits.
  *
- *  O [M, d_model] gated context; W_o [d_model, d_model]; Y [M, d_model].
- *  workspace >= gmla_gate_out_workspace_size(M, d_model) bytes.
+ *  O [M, d_model] context; G [M, d_model] gate logits or NULL;
+ *  W_o [d_model, d_model]; Y [M, d_model] output.
+ *  workspace: with G != NULL, >= gmla_gate_out_workspace_size(M, d_model)
+ *          bytes, 16-byte aligned; it receives the gated context (bfloat16)
+ *          that the projection then reads.  With G == NULL it is not used
+ *          and may be NULL.
+ * Errors: GMLA_ERR_ARG for null or misaligned pointers; GMLA_ERR_UNSUPPORTED
+ * when d_model is not a multiple of 128; GMLA_ERR_WORKSPACE for a missing or
+ * short workspace when G is given.
  */
 GMLA_API gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M,
                           int64_t d_model, gmla_bf16 *Y, void *workspace, size_t workspace_bytes,
                           gmla_stream_t stream);
 GMLA_API size_t gmla_gate_out_workspace_size(int64_t M, int64_t d_model);
+
+/*
+ * gmla_gate_out_heads -- the share of the heads [head_begin, head_end) in
+ * gmla_gate_out: Y_part = (sigmoid(G) (.) O) W_o[:, c]^T with c the channels
+ * 128*head_begin .. 128*head_end - 1.  The output projection mixes all
+ * channels, so Y is the sum of the shares of any partition of the heads
+ * (each GPU of a head-parallel layer computes its share; a reduction over
+ * the GPUs gives Y).
+ *
+ *  O, G    [M, 128 * (head_end - head_begin)]: the context and gate logits of
+ *          the range (G may be NULL)
+ *  W_o     the FULL [d_model, d_model] weight (only the range's columns are read)
+ *  Y       [M, d_model] output: this range's share
+ *  workspace: with G != NULL, >= gmla_gate_out_workspace_size(M,
+ *          128 * (head_end - head_begin)) bytes.
+ *  0 <= head_begin < head_end <= d_model / 128; errors as gmla_gate_out.
+ */
+GMLA_API gmla_status gmla_gate_out_heads(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M,
+                                        int64_t d_model, int64_t head_begin, int64_t head_end, gmla_bf16 *Y,
+                                        void *workspace, size_t workspace_bytes, gmla_stream_t stream);
 
 /* Synchronise `stream`, then read and clear this device's status word.
  * Returns GMLA_OK, GMLA_ERR_TIMEOUT (a bounded wait ran out) or GMLA_ERR_CUDA. */

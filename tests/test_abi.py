@@ -78,11 +78,17 @@ def test_host_validation_without_gpu(gmla):
                                  None) == 2
     # latent project: cache too short, K requested without C, d_model not a multiple of 128
     assert L.gmla_latent_project(fake, 2, 10, 256, fake, fake, fake, 64, fake, fake, fake, fake, fake, 15, 6, None,
-                                 None, None, 0, None) == 1
+                                 None, None) == 1
     assert L.gmla_latent_project(fake, 2, 10, 256, fake, fake, fake, 64, fake, fake, fake, fake, None, 16, 0, fake,
-                                 None, None, 0, None) == 1
+                                 None, None) == 1
     assert L.gmla_latent_project(fake, 2, 10, 200, fake, fake, fake, 64, fake, fake, fake, fake, fake, 16, 0, None,
-                                 None, None, 0, None) == 2
+                                 None, None) == 2
+    # head-range projections: empty range, range past the heads
+    LPH = L.gmla_latent_project_heads
+    assert LPH(fake, 2, 10, 256, 1, 1, fake, fake, fake, 64, fake, fake, fake, fake, fake, 16, 0, None, None,
+               None) == 1
+    assert LPH(fake, 2, 10, 256, 1, 3, fake, fake, fake, 64, fake, fake, fake, fake, fake, 16, 0, None, None,
+               None) == 1
     # decode: L beyond the cache, and a short workspace
     assert L.gmla_attend_decode(fake, fake, 2, 100, 101, 2, 128, 64, fake, fake, 0.0, None, fake, None, fake, 1 << 30,
                                 None) == 1
@@ -125,9 +131,26 @@ def test_host_validation_without_gpu(gmla):
     # the timeout self-test refuses limits outside 1..1000 ms
     assert L.gmla_selftest_wait_timeout(0, None) == 1
     assert L.gmla_selftest_wait_timeout(5000, None) == 1
-    # gate_out: the gate is fused upstream
-    assert L.gmla_gate_out(fake, fake, fake, 4, 256, fake, None, 0, None) == 2
+    # gate_out: a gate needs a workspace for the gated context; bad pointers and head ranges
+    assert L.gmla_gate_out(fake, fake, fake, 4, 256, fake, None, 0, None) == 5
+    need = L.gmla_gate_out_workspace_size(4, 256)
+    assert need >= 4 * 256 * 2
+    assert L.gmla_gate_out(fake, fake, fake, 4, 256, fake, fake, need - 1, None) == 5
     assert L.gmla_gate_out(None, None, fake, 4, 256, fake, None, 0, None) == 1
+    assert L.gmla_gate_out(fake, None, fake, 4, 200, fake, None, 0, None) == 2
+    assert L.gmla_gate_out_heads(fake, None, fake, 4, 256, 0, 3, fake, None, 0, None) == 1
+    assert L.gmla_gate_out_heads(fake, None, fake, 4, 256, 2, 1, fake, None, 0, None) == 1
+    # partial decode: bad key ranges, a short workspace; combine: no parts, too many parts
+    PD = L.gmla_attend_decode_partial
+    assert PD(fake, fake, 2, 100, 50, 40, 2, 128, 64, fake, 0.0, fake, fake, fake, 1 << 30, None) == 1
+    assert PD(fake, fake, 2, 100, 0, 101, 2, 128, 64, fake, 0.0, fake, fake, fake, 1 << 30, None) == 1
+    assert PD(fake, fake, 2, 100, 10, 60, 2, 128, 64, fake, 0.0, fake, fake, fake, 16, None) == 5
+    assert PD(fake, fake, 2, 100, 10, 60, 2, 128, 64, fake, 0.0, None, fake, fake, 1 << 30, None) == 1
+    assert L.gmla_attend_decode_partial_workspace_size(2, 10, 60, 2, 64) > 16
+    assert L.gmla_attend_decode_partial_workspace_size(2, 10, 10, 2, 64) == 0
+    assert L.gmla_decode_combine(fake, fake, 0, 2, 2, 128, 64, fake, None, fake, None) == 1
+    assert L.gmla_decode_combine(fake, fake, 1025, 2, 2, 128, 64, fake, None, fake, None) == 2
+    assert L.gmla_decode_combine(fake, fake, 2, 2, 2, 128, 96, fake, None, fake, None) == 2
 
 
 def test_binding_has_no_cpu_path():

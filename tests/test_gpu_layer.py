@@ -65,6 +65,111 @@ def test_gate_out_matches_oracle(g):
     assert_parity(f64(Y), orc.linear(O, W), "Y")
 
 
+def test_gate_out_with_gate_matches_oracle(g):
+    """gmla_gate_out given the gate logits: Y = (sigmoid(G) (.) O) W_o^T, the gate
+    before W_o ("Gated MLA" page, "The channel-wise output gate"); logits of -inf
+    close every channel, so Y is exactly 0 there."""
+    rng = np.random.default_rng(5)
+    from synth_inputs import bf16_bits_from_f64
+    M, d = 300, 384
+    O = bf16_bits_from_f64(rng.standard_normal((M, d)))
+    Gl = bf16_bits_from_f64(rng.standard_normal((M, d)))
+    Gl[17] = 0xFF80  # bfloat16 -inf: row 17 fully gated off
+    W = bf16_bits_from_f64(rng.standard_normal((d, d)) / np.sqrt(d))
+    Y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    work = ws(g.gmla_gate_out_workspace_size(M, d))
+    g.gmla_gate_out(to_dev(O), to_dev(W), Y, G=to_dev(Gl), workspace=work)
+    g.gmla_get_device_status()
+    ref = orc.linear(orc.gate(O, Gl), W)
+    assert np.all(ref[17] == 0)
+    got = f64(Y)
+    assert np.all(got[17] == 0)
+    assert_parity(got, ref, "gated Y")
+    # without its workspace the gated form is refused before any launch
+    assert g.STATUS[g.gmla_gate_out(to_dev(O), to_dev(W), Y, G=to_dev(Gl), check=False)] == "GMLA_ERR_WORKSPACE"
+
+
+def test_gemm_persistent_multi_tile_full_output(g):
+    """More than 2 x 148 output tiles per launch, so every CTA of the persistent
+    GEMM runs three or four tiles: both TMEM accumulators, the phase flips of
+    their barriers across tiles and several groups of the grouped raster are
+    exercised, and every output element is compared with the oracle."""
+    B, T, H, d_c = 2, 2048, 12, 512
+    d = 128 * H
+    w, t = make_layer(41, B, T, d, d_c)
+    Q = torch.empty(B, T, d, dtype=torch.bfloat16, device="cuda")
+    G, K, V = (torch.empty_like(Q) for _ in range(3))
+    C = torch.empty(B, T, d_c, dtype=torch.bfloat16, device="cuda")
+    # [Q | G | C]: 32 m-tiles x (6 + 6 + 2) n-tiles = 448 tiles; [K | V]: 32 x 12 = 384 tiles
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=Q, G=G, C=C, K=K, V=V)
+    # W_o with the gate: 64 m-tiles x 6 n-tiles = 384 tiles
+    dr = Draw(43)
+    O2, G2 = dr.normal((8192, d)), dr.normal((8192, d))
+    Y2 = torch.empty(8192, d, dtype=torch.bfloat16, device="cuda")
+    g.gmla_gate_out(to_dev(O2), t["W_o"], Y2, G=to_dev(G2), workspace=ws(g.gmla_gate_out_workspace_size(8192, d)))
+    g.gmla_get_device_status()
+    assert_parity(f64(Q), orc.linear(w["X"], w["W_q"]), "Q (448 tiles)")
+    assert_parity(f64(G), orc.linear(w["X"], w["W_g"]), "G (448 tiles)")
+    Cref = orc.linear(w["X"], w["W_c"])
+    assert_parity(f64(C), Cref, "C (448 tiles)")
+    Cr = orc.round_bf16(Cref)
+    assert_parity(f64(K), orc.linear(Cr, w["W_k"]), "K (384 tiles)")
+    assert_parity(f64(V), orc.linear(Cr, w["W_v"]), "V (384 tiles)")
+    assert_parity(f64(Y2), orc.linear(orc.gate(O2, G2), w["W_o"]), "gated W_o (384 tiles)")
+
+
+def test_layer_full_size_sampled_rows(g):
+    """The full layer at its prefill size -- B=2, T=4096, d_model=12288 (96 heads of
+    128), d_c=512 -- through the C ABI: gmla_latent_project (Q, G, C, K, V),
+    gmla_attend_prefill with the gate, gmla_gate_out.  The GEMMs run 12416, 12288
+    and 6144 tiles on 148 CTAs.  Checked at 32 token rows spread over both
+    sequences and all four 16-m-tile raster groups, against the oracle, which
+    rounds to bfloat16 where the library stores bfloat16 ("Gated MLA" page,
+    "Implementation order")."""
+    B, T, H, d_c = 2, 4096, 96, 512
+    d = 128 * H
+    w, t = make_layer(SEEDS["layer_prefill"], B, T, d, d_c)
+    Q = torch.empty(B, T, d, dtype=torch.bfloat16, device="cuda")
+    G, K, V, O, Y = (torch.empty_like(Q) for _ in range(5))
+    C = torch.empty(B, T, d_c, dtype=torch.bfloat16, device="cuda")
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=Q, G=G, C=C, K=K, V=V)
+    v4 = lambda x: x.view(B, T, H, 128)
+    g.gmla_attend_prefill(v4(Q), v4(K), v4(V), v4(O), G=G)
+    g.gmla_gate_out(O, t["W_o"], Y)
+    g.gmla_get_device_status()
+    del t
+    torch.cuda.empty_cache()
+
+    rng = np.random.default_rng(4)
+    m_tiles = np.concatenate([rng.choice(np.arange(q * 16, q * 16 + 16), 8, replace=False) for q in range(4)])
+    rows = np.sort(m_tiles * 128 + rng.integers(0, 128, m_tiles.size))  # flat token rows in [0, B*T)
+    rb = orc.round_bf16
+    X2 = w["X"].reshape(B * T, d)
+    flat = lambda x: f64(x).reshape(B * T, -1)[rows]
+    # per-step checks on the sampled rows
+    Qref = orc.linear(X2, w["W_q"], rows=rows)[rows]
+    assert_parity(flat(Q), Qref, "Q rows")
+    Gref = orc.linear(X2, w["W_g"], rows=rows)[rows]
+    assert_parity(flat(G), Gref, "G rows")
+    Call = orc.linear(X2, w["W_c"])                                  # every row: keys and values need them
+    assert_parity(flat(C), Call[rows], "C rows")
+    Kall = orc.linear(rb(Call), w["W_k"])
+    Vall = orc.linear(rb(Call), w["W_v"])
+    assert_parity(flat(K), Kall[rows], "K rows")
+    assert_parity(flat(V), Vall[rows], "V rows")
+    # chained: attention of the sampled rows over the oracle's own bf16-rounded K, V
+    Qfull = np.zeros((B * T, d))
+    Qfull[rows] = rb(Qref)
+    trip = np.array([(r // T, h, r % T) for r in rows for h in range(H)], dtype=np.int64)
+    Oh = orc.attention(Qfull.reshape(B, T, H, 128), rb(Kall).reshape(B, T, H, 128), rb(Vall).reshape(B, T, H, 128),
+                       rows=trip)
+    Og = rb(orc.gate(Oh.reshape(B * T, d)[rows], rb(Gref)))
+    assert_parity(flat(O), Og, "gated context rows")
+    Ofull = np.zeros((B * T, d))
+    Ofull[rows] = Og
+    assert_parity(flat(Y), orc.linear(Ofull, w["W_o"], rows=rows)[rows], "Y rows")
+
+
 def test_layer_chained_matches_oracle(g):
     """X -> projections -> attention (+ gate) -> W_o, against the oracle that rounds
     to bfloat16 at the same library boundaries."""

@@ -14,8 +14,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as orc
 from synth_inputs import Draw
-from tests.gpu_util import assert_parity, f64, to_dev
+from tests.gpu_util import ROW_SUM, assert_parity, f64, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +44,31 @@ def test_noalloc_decode_matches_workspace_decode_on_consecutive_calls():
         g.gmla_attend_decode_noalloc(Q, C, L, Wk, Wv, out, H, G=G)
         g.gmla_get_device_status()
         assert_parity(f64(out), f64(ref), f"no-alloc vs workspace decode, B={B} L={L}")
+        # the no-alloc call may split the keys differently, so it is also held to the
+        # oracle's plain decode (K and V rebuilt from the cache) on sampled heads
+        pairs = [(0, 0), (B - 1, H - 1), (B // 2, 17)]
+        oref = orc.decode_latent(x["q"], x["cache"], L, x["Wk"], x["Wv"], H, G=x["G"], heads=pairs)
+        sel = np.concatenate([np.arange(h * 128, (h + 1) * 128) + b * d for b, h in pairs])
+        assert_parity(f64(out).reshape(-1)[sel], oref.reshape(-1)[sel], f"no-alloc vs oracle, B={B} L={L}")
+
+
+def test_noalloc_decode_debug_weights():
+    """The debug softmax weights of the no-alloc call (normalised through the
+    log-sum-exp kept in the shared scratch): rows sum to one and match the
+    oracle's weights."""
+    import causal_head_latent_b200 as g
+    B, L, Lmax, H, d_c = 2, 777, 800, 4, 512
+    x = _inputs(702, B, Lmax, H, d_c)
+    Q, C, Wk, Wv, G = (to_dev(x[k]) for k in ("q", "cache", "Wk", "Wv", "G"))
+    out = torch.empty(B, 128 * H, dtype=torch.bfloat16, device="cuda")
+    W = torch.full((B, H, L), float("nan"), device="cuda")
+    g.gmla_attend_decode_noalloc(Q, C, L, Wk, Wv, out, H, G=G, weights=W)
+    g.gmla_get_device_status()
+    w = f64(W)
+    assert np.abs(w.sum(-1) - 1.0).max() <= ROW_SUM
+    ref, wref = orc.decode_latent(x["q"], x["cache"], L, x["Wk"], x["Wv"], H, G=x["G"], want_weights=True)
+    assert_parity(f64(out), ref, "no-alloc decode with weights")
+    assert np.all(np.abs(w - wref) <= 2e-5 + 1e-2 * wref)
 
 
 def test_noalloc_decode_refuses_problems_beyond_its_scratch():
