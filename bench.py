@@ -1,20 +1,26 @@
 """Benchmark of the Gated MLA hot path on B200.
 
-One step = one pass of the hot path over one synthetic batch:
+One step = one pass of the whole hot path, every step of the method, over one
+synthetic batch of each workload shape:
   prefill  causal attention, B=1, 96 heads, T=8192, D_h=128 (gmla_attend_prefill)
   decode   one new token for B=32 sequences over L=131072 cached latents of width
            512: projections of the new token with the latent appended at row
            L-1 (gmla_latent_project), absorbed attention over the latent cache
            with log-sum-exp combine and gate (gmla_attend_decode), W_o
            (gmla_gate_out); d_model = 12288.
+  plain    decode attention over explicit K, V in the "Softmax over keys" page's
+           shape: B=8, 96 heads, one query, 1001 keys (gmla_attend_prefill, Tq=1)
+  layer    the full layer prefill, B=2, T=4096, d_model=12288, d_c=512:
+           projections with K/V expansion, gated causal attention, W_o.
 Headline value: prefill attention TFLOP/s (causal pairs only:
 4*D_h*H*B*T(T+1)/2 flop).  The decode half of the metric -- latent-cache GB/s
-of gmla_attend_decode -- is reported in the "decode" object.  Both inputs are
-larger than L2 (Q/K/V 604 MB, cache 4.3 GB), so no flush is needed between
-steps.
+of gmla_attend_decode -- is reported in the "decode" object, the other two
+workloads in "decode_plain" and "layer".  Every input but the plain decode's
+is larger than L2 (Q/K/V 604 MB, cache 4.3 GB, layer weights 0.9 GB); the
+plain decode (394 MB) runs after the others, which evict it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--parts all|prefill|decode] [--workload step|layer]
+                    [--parts all|prefill|decode|plain|layer] [--workload step|layer|sweep|varlen]
 
 With --gpus N > 1 (launched by torch.distributed.run) every rank runs the same
 per-GPU workload (data-parallel replicas, no collective on the data path);
@@ -56,6 +62,14 @@ VL_KV = (8192, 8192, 6000, 1024, 8192, 4096, 3000, 5000)
 VL_DEC_B, VL_DEC_LMAX = 32, 131072
 
 
+PL_B, PL_TK = 8, 1001  # plain decode over explicit K, V (the "Softmax over keys" page, p = 1000)
+
+
+def plain_decode_bytes(B=PL_B, H=96, Tk=PL_TK):
+    # Q, K, V and O of gmla_attend_prefill with one query
+    return 2.0 * B * H * D * (2 * Tk + 2)
+
+
 def prefill_flops(B=P_B, H=P_H, T=P_T):
     return 4.0 * D * H * B * T * (T + 1) / 2
 
@@ -80,26 +94,31 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant kernels,
-# from one ncu capture each (profiles/).  Reported only while the kernel source is the one that
-# was captured (sha1 of the file); any change makes it null until the next capture.
+# from one ncu capture each (profiles/).  Reported only while the kernel sources are the ones that
+# were captured (sha1 over the listed files, in order); any change makes it null until the next
+# capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill.cu": {"sha1": "ffe545376afcfed7e56882a64169aa1db2a810c1", "bytes": 604.147456e6 + 183.511808e6,
-                        "how": "ncu capture at the timed size (B=1 H=96 T=8192)"},
-    "attn_latent_tc.cu": {"sha1": "4e8f5fb90ca5916411bfc57aec6f7184683f8cb9", "bytes": 543.840256e6 * 8 + 32.554752e6,
-                          "how": "ncu capture of latent_decode_kernel at L=16384, reads scaled x8 to L=131072 (cache "
-                                 "traffic grows with L), partial-state writes unscaled"},
+    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": None, "bytes": None, "how": None},
+    "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu"], "sha1": None, "bytes": None,
+                           "how": None},
 }
 
 
-def profiled_traffic(src):
+def sources_sha1(files):
     import hashlib
-    ent = PROFILED_TRAFFIC.get(src)
-    path = os.path.join(ROOT, "causal_head_latent_b200", "csrc", src)
-    if not ent or not os.path.exists(path):
-        return None, None
-    with open(path, "rb") as f:
-        if hashlib.sha1(f.read()).hexdigest() != ent["sha1"]:
-            return None, "kernel changed since the ncu capture"
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, "causal_head_latent_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel):
+    ent = PROFILED_TRAFFIC.get(kernel)
+    if not ent or ent["bytes"] is None:
+        return None, "no ncu capture of the current source"
+    if sources_sha1(ent["sources"]) != ent["sha1"]:
+        return None, "kernel changed since the ncu capture"
     return ent["bytes"], ent["how"]
 
 
@@ -117,13 +136,17 @@ def load_peaks():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock and throttle-reason samples every 50 ms, each with the host
+    time it was taken, so that a summary can be cut for any timed region."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.samples = []  # (host time, sm MHz, max MHz, set of active reasons)
 
     def start(self):
         try:
@@ -135,29 +158,40 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        import datetime
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                t = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(f[2]), float(f[3])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            self.samples.append((t, sm, mx, {n for n, v in zip(self.NAMES, f[6:10]) if v.lower().startswith("active")}))
+
+    def summary(self, t0=None, t1=None):
+        """Median SM clock, max clock and active reasons of the samples in [t0, t1]
+        (host time); a region shorter than the sampling period takes the samples
+        nearest to it."""
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sel = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        if not sel and self.samples and t0 is not None:
+            mid = 0.5 * (t0 + t1)
+            near = sorted(self.samples, key=lambda x: abs(x[0] - mid))[:2]
+            sel = [x for x in near if abs(x[0] - mid) < 0.2]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(x[1] for x in sel), "sm_max_mhz": max(x[2] for x in sel),
+                "reasons": sorted(set().union(*(x[3] for x in sel))), "samples": len(sel)}
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -261,7 +295,7 @@ class DecodePart:
         self.ws_d = torch.empty(g.gmla_attend_decode_workspace_size(DEC_B, DEC_L, DM // D, DC), dtype=torch.uint8,
                                 device="cuda")
         self.bytes = decode_bytes()
-        self.launches = 6
+        self.launches = 5  # projection GEMM, absorb, latent stream, combine, W_o GEMM
 
     def project(self):
         import causal_head_latent_b200 as g
@@ -286,6 +320,24 @@ class DecodePart:
         self.Y_host.copy_(self.Y, non_blocking=True)
 
 
+class PlainDecodePart:
+    """Decode attention over explicit K, V: B=8, 96 heads, one query at position
+    1000 over 1001 keys, [B, H, T, D] layout (the "Softmax over keys" page)."""
+
+    def __init__(self, seed):
+        import torch
+        from synth_inputs import decode_plain_qkv
+        inp = decode_plain_qkv(seed, PL_B, 96, PL_TK)
+        self.Q, self.K, self.V = (dev(inp[k]) for k in ("Q", "K", "V"))
+        self.O = torch.empty_like(self.Q)
+        self.bytes = plain_decode_bytes()
+        self.launches = 1
+
+    def run(self):
+        import causal_head_latent_b200 as g
+        g.gmla_attend_prefill(self.Q, self.K, self.V, self.O, causal=True, layout="bhtd")
+
+
 class LayerPart:
     """Full Gated MLA layer prefill: B=2, T=4096, d_model=12288, d_c=512."""
 
@@ -298,17 +350,28 @@ class LayerPart:
         self.G, self.K, self.V, self.O, self.Y = (torch.empty_like(self.Q) for _ in range(5))
         self.C = torch.empty(L_B, L_T, DC, dtype=torch.bfloat16, device="cuda")
         self.flops = layer_flops()
-        self.launches = 4
+        self.launches = 4  # [Q|G|C] GEMM, [K|V] GEMM, attention, W_o GEMM
 
-    def run(self):
+    def project(self):
         import causal_head_latent_b200 as g
         t = self.t
-        H = DM // D
         g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], t["W_k"], t["W_v"], Q=self.Q, G=self.G, C=self.C,
                               K=self.K, V=self.V)
+
+    def attend(self):
+        import causal_head_latent_b200 as g
+        H = DM // D
         v = lambda x: x.view(L_B, L_T, H, D)
         g.gmla_attend_prefill(v(self.Q), v(self.K), v(self.V), v(self.O), G=self.G)
-        g.gmla_gate_out(self.O, t["W_o"], self.Y)
+
+    def out(self):
+        import causal_head_latent_b200 as g
+        g.gmla_gate_out(self.O, self.t["W_o"], self.Y)
+
+    def run(self):
+        self.project()
+        self.attend()
+        self.out()
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
@@ -400,9 +463,10 @@ def config_obj(args):
                 "l2": "inputs larger than L2"}
     return {"workload": f"causal prefill attention B={P_B} H={P_H} T={P_T} D_h={D} bf16 + latent-cache decode "
                         f"B={DEC_B} L={DEC_L} d_c={DC} H=96 d_model={DM} (projections, append, absorbed attention, "
-                        f"LSE combine, gate, W_o)",
+                        f"LSE combine, gate, W_o) + decode over explicit K/V B={PL_B} H=96 Tk={PL_TK} + full layer "
+                        f"prefill B={L_B} T={L_T} d_model={DM} d_c={DC}",
             "global_batch": P_B * max(1, args.gpus), "seq_len": P_T, "parallelism": f"dp{args.gpus}",
-            "parts": args.parts, "l2": "inputs larger than L2 (Q/K/V 604 MB, cache 4.3 GB); no flush"}
+            "parts": args.parts, "l2": "inputs larger than L2 (Q/K/V 604 MB, cache 4.3 GB, layer 2.4 GB); no flush"}
 
 
 def timed(fn_list, steps, world):
@@ -466,7 +530,8 @@ def run_varlen(args, rank, world, local, peaks):
     clk = ClockSampler(local)
     clk.start()
     total, per = timed([fp, fd], args.steps, world)
-    clocks = clk.stop()
+    clk.stop()
+    clocks = clk.summary()
     g.gmla_get_device_status()
     total = max_over_ranks(total, world)
     p_ms = max_over_ranks(per[0], world) / args.steps
@@ -547,7 +612,8 @@ def run_sweep(args, rank, world, local, peaks):
                      "decode_ms": d_ms, "decode_gbs": db / (d_ms / 1e3) / 1e9,
                      "decode_frac_of_hbm": db / (d_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                      "cache_bytes_per_sequence": T * DC * 2})
-    clocks = clk.stop()
+    clk.stop()
+    clocks = clk.summary()
     ratios = {}
     for a, b in ((0, 1), (1, 2)):
         ta, tb = SWEEP_T[a], SWEEP_T[b]
@@ -576,7 +642,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--parts", default="all", choices=["all", "prefill", "decode"])
+    ap.add_argument("--parts", default="all", choices=["all", "prefill", "decode", "plain", "layer"])
     ap.add_argument("--workload", default="step", choices=["step", "layer", "sweep", "varlen"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
@@ -612,7 +678,8 @@ def main():
         clk = ClockSampler(local)
         clk.start()
         total, per = timed([part.run], args.steps, world)
-        clocks = clk.stop()
+        clk.stop()
+        clocks = clk.summary()
         g.gmla_get_device_status()
         total = max_over_ranks(total, world)
         val = part.flops * args.steps * world / (total / 1e3) / 1e12
@@ -629,71 +696,130 @@ def main():
             print(json.dumps(line), flush=True)
         return
 
-    parts = []
-    pre = dec = None
+    pre = dec = plain = layer = None
     if args.parts in ("all", "prefill"):
         pre = PrefillPart(3)
     if args.parts in ("all", "decode"):
         dec = DecodePart(5)
-    fns, names = [], []
+    if args.parts in ("all", "layer"):
+        layer = LayerPart(4)
+    if args.parts in ("all", "plain"):
+        plain = PlainDecodePart(2)
+    # One step is one pass over every workload.  Each workload is warmed up and
+    # timed in a region of its own (K steps), in this order, so that the power
+    # drawn by the GEMM-heavy full layer does not lower the clock of the kernels
+    # measured before it; each region reports the clocks sampled during it.
+    regions = []
     if pre:
-        fns.append(pre.run)
-        names.append("prefill_attention")
+        regions.append(("prefill", [("prefill_attention", pre.run)]))
     if dec:
-        fns += [dec.project, dec.attend, dec.out]
-        names += ["decode_project", "decode_attend", "decode_out"]
-
-    for _ in range(args.warmup):
-        for fn in fns:
-            fn()
-    g.gmla_get_device_status()
-
+        regions.append(("decode", [("decode_project", dec.project), ("decode_attend", dec.attend),
+                                   ("decode_out", dec.out)]))
+    if plain:
+        regions.append(("plain", [("plain_decode", plain.run)]))
+    if layer:
+        regions.append(("layer", [("layer_project", layer.project), ("layer_attend", layer.attend),
+                                  ("layer_out", layer.out)]))
+    K = args.steps
     clk = ClockSampler(local)
     clk.start()
-    total, per = timed(fns, args.steps, world)
-    clocks = clk.stop()
-    g.gmla_get_device_status()
-    total = max_over_ranks(total, world)
-    per = [max_over_ranks(p, world) for p in per]
-    perd = dict(zip(names, per))
-    K = args.steps
-    launches = (1 if pre else 0) + (dec.launches if dec else 0)
+    time.sleep(0.3)  # the sampler's first sample
+    perd, region_ms, region_clocks = {}, {}, {}
+    for rname, fl in regions:
+        for _ in range(args.warmup):
+            for _, fn in fl:
+                fn()
+        g.gmla_get_device_status()
+        h0 = time.time()
+        rt, per = timed([fn for _, fn in fl], K, world)
+        h1 = time.time()
+        g.gmla_get_device_status()
+        region_ms[rname] = max_over_ranks(rt, world)
+        region_clocks[rname] = (h0, h1)
+        for (n, _), v in zip(fl, per):
+            perd[n] = max_over_ranks(v, world)
+    time.sleep(0.1)
+    clk.stop()
+    t_first, t_last = min(h[0] for h in region_clocks.values()), max(h[1] for h in region_clocks.values())
+    region_clocks = {r: clk.summary(*hh) for r, hh in region_clocks.items()}
+    clocks = clk.summary(t_first, t_last)  # every timed region, warm-ups between them included
+    total = sum(region_ms.values())
+    launches = sum(p.launches for p in (pre, dec, layer, plain) if p is not None)
+    # the prefill region is tens of milliseconds at the sampled clock: the burst
+    # peak (a short cuBLAS run) is its denominator; the sustained one (seconds
+    # under the power cap) is reported beside it
+    burst = peaks["bf16_tflops"]
 
     line = {"metric": METRIC, "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_obj(args), "clocks": clocks, "gpu_launches": launches * K,
-            "kernel_ms_per_step": {k: v / K for k, v in perd.items()}}
+            "kernel_ms_per_step": {k: v / K for k, v in perd.items()},
+            "regions": {r: {"ms_per_step": region_ms[r] / K, "clocks": region_clocks[r]} for r in region_ms}}
     if pre:
         t_att = perd["prefill_attention"] / K
         val = pre.flops * world / (t_att / 1e3) / 1e12
         line.update(value=val, unit="TFLOP/s")
         ach = pre.flops / (t_att / 1e3) / 1e12
-        line["roofline"] = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"],
-                            "traffic": profiled_traffic("attn_prefill.cu")[0],
-                            "traffic_source": profiled_traffic("attn_prefill.cu")[1],
+        tr, tr_how = profiled_traffic("attn_prefill_kernel")
+        line["roofline"] = {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s",
+                            "frac": ach / burst, "traffic": tr, "traffic_source": tr_how,
                             "algorithmic_bytes": 2.0 * 4 * P_B * P_T * P_H * D,
                             "kernel": "attn_prefill_kernel",
-                            "peak_kind": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)",
-                            "frac_of_burst": ach / peaks["bf16_tflops"], "frac_of_datasheet_2250": ach / 2250.0}
+                            "peak_kind": f"{peaks['source']} burst bf16 (timed region of {region_ms['prefill']:.0f} ms "
+                                         f"at {region_clocks['prefill']['sm_mhz']} MHz)",
+                            "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
+                            "frac_of_datasheet_2250": ach / 2250.0}
     if dec:
         t_dec = perd["decode_attend"] / K
         gbs = dec.bytes / (t_dec / 1e3) / 1e9
         t_step = (perd["decode_project"] + perd["decode_attend"] + perd["decode_out"]) / K
+        tr, tr_how = profiled_traffic("gmla_attend_decode") if DEC_L == 131072 else (None, None)
         dobj = {"value": gbs * world, "unit": "GB/s", "ms_per_step": t_dec,
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": gbs / peaks["hbm_gbs"],
-                             "traffic": profiled_traffic("attn_latent_tc.cu")[0] if DEC_L == 131072 else None,
-                             "traffic_source": profiled_traffic("attn_latent_tc.cu")[1],
-                             "kernel": "gmla_attend_decode",
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": tr, "traffic_source": tr_how,
+                             "algorithmic_bytes": dec.bytes, "kernel": "gmla_attend_decode",
                              "peak_kind": f"{peaks['source']} HBM copy", "frac_of_datasheet_8000": gbs / 8000.0},
-                "step_ms": t_step, "step_gbs": decode_step_bytes() / (t_step / 1e3) / 1e9}
+                "step_ms": t_step, "step_gbs": decode_step_bytes() / (t_step / 1e3) / 1e9,
+                "workload": f"latent-cache decode B={DEC_B} L={DEC_L} d_c={DC} H=96 d_model={DM}",
+                "clocks": region_clocks["decode"]}
         line["decode"] = dobj
         if not pre:
             line.update(value=gbs * world, unit="GB/s", roofline=dobj["roofline"])
+    if layer:
+        t_l = sum(perd[k] for k in ("layer_project", "layer_attend", "layer_out")) / K
+        tf = layer.flops / (t_l / 1e3) / 1e12
+        H = DM // D
+        M = L_B * L_T
+        parts_flops = {"layer_project": 2.0 * M * DM * (2 * DM + DC) + 2.0 * M * DC * 2 * DM,
+                       "layer_attend": prefill_flops(L_B, H, L_T), "layer_out": 2.0 * M * DM * DM}
+        lobj = {"value": tf * world, "unit": "TFLOP/s", "ms_per_step": t_l,
+                "workload": f"Gated MLA layer prefill B={L_B} T={L_T} d_model={DM} H=96 D_h=128 d_c={DC}",
+                "algorithmic_flops": layer.flops,
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": burst, "unit": "TFLOP/s", "frac": tf / burst,
+                             "traffic": None, "peak_kind": f"{peaks['source']} burst bf16",
+                             "frac_of_sustained": tf / peaks["bf16_tflops_sustained"]},
+                "clocks": region_clocks["layer"],
+                "calls": {k: {"ms": perd[k] / K, "tflops": f / (perd[k] / K / 1e3) / 1e12}
+                          for k, f in parts_flops.items()}}
+        line["layer"] = lobj
+        if not (pre or dec):
+            line.update(value=tf * world, unit="TFLOP/s", roofline=lobj["roofline"])
+    if plain:
+        t_p = perd["plain_decode"] / K
+        gbs = plain.bytes / (t_p / 1e3) / 1e9
+        pobj = {"value": gbs * world, "unit": "GB/s", "ms_per_step": t_p,
+                "workload": f"decode attention over explicit K/V B={PL_B} H=96 Tq=1 Tk={PL_TK} D_h=128 [B,H,T,D]",
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": plain.bytes,
+                             "kernel": "attn_rows_kernel", "peak_kind": f"{peaks['source']} HBM copy",
+                             "l2": "394 MB of K/V, timed back to back (a step reads them once; about 3x L2)"},
+                "clocks": region_clocks["plain"]}
+        line["decode_plain"] = pobj
+        if not (pre or dec or layer):
+            line.update(value=gbs * world, unit="GB/s", roofline=pobj["roofline"])
 
     # end-to-end through the public API with pinned host buffers
-    if not args.no_e2e:
+    if not args.no_e2e and (pre or dec):
         ke = max(1, min(K, 5))
         if pre:
             for _ in range(1):

@@ -4,9 +4,9 @@
 // online-softmax state for all H (<= 96) heads at once; every latent tile is
 // read from HBM once and used twice, as keys and as values:
 //   S      [head, key]  = q~ C_tile^T          M=128 (heads, zero-padded by
-//                                               overlap), N=48 keys, K=d_c
+//                                               overlap), N=KT keys, K=d_c
 //   acc^T  [d_c, head] += C_tile^T P^T^T       M=128 per d_c block, N=96 heads,
-//                                               K=48 keys (C tile read MN-major)
+//                                               K=KT keys (C tile read MN-major)
 // with P^T [head, key] = 2^(S - m_head) in shared memory.  q~ = scale*log2(e) *
 // W_k^(h)T q_h comes from the absorb kernel (bfloat16), so S is already in
 // the exp2 domain.  P is rounded to bfloat16 before it multiplies the
@@ -17,25 +17,30 @@
 //  * an SM takes in at most ~22.5 bytes per cycle through TMA, from L2 as
 //    from HBM, so the 1 KB latent row of a key costs >= 45 cycles of ingress
 //    and the latent stream has to stay in flight without gaps;
-//  * a tcgen05.mma with N <= 128 costs ~66 cycles whatever its M and N, so the
-//    MMA count per key sets the compute floor: 32 score + 12 value MMAs per
-//    48-key tile, ~61 cycles per key;
+//  * a tcgen05.mma with N <= 128 costs ~56-66 cycles whatever its M and N, so
+//    the MMA count per key sets the compute floor: 32 score MMAs per tile
+//    (d_c / 16, whatever KT) and 4 value MMAs per 16 keys;
 //  * the MMA-issuing thread must not stall: a wait on its own recent MMAs
 //    (through a barrier and another warp) drains the MMA pipe, an acquire
 //    mbarrier wait between small MMAs costs ~270 cycles even when the phase
 //    has completed (a relaxed poll plus fence.acq_rel costs ~90), and each
 //    tcgen05.commit ~95.
-// Hence 48-key tiles: an 18-chunk latent ring (2.25 tiles) lets the loads of
-// tile j stream while tiles j-1 and j-2 are still in use; S is double-
-// buffered in TMEM so the score MMAs of the next tile never wait for the
-// softmax; the score and value MMAs come from two threads, so the value MMAs
-// of a tile go out as soon as its probabilities are ready (releasing ring
-// slots for tile j+2 early) while score MMAs keep the pipe busy; and the ring
-// moves in chunk pairs, so a tile costs the score thread three waits and one
-// commit and the value thread one wait and two commits.
+// Tiles of KT = 48 keys (kLatentTileKeys; 64 also builds): 0.92 MMAs per key,
+// and an 18-chunk latent ring (2.25 tiles) next to the 96 KB of q~, so every
+// load of tile j reuses a slot of tile j-2 or j-3 and streams while tiles
+// j-1 and j-2 are still in use.  64-key tiles need only 0.75 MMAs per key, but
+// their 14-chunk ring (1.75 tiles: shared memory is full) makes the last chunk
+// pair of tile j wait for the value MMAs of tile j-1, which measured slower.
+// S is double-buffered in TMEM (2 x 64 columns next to the 384 of acc^T), so
+// the score MMAs of the next tile never wait for the softmax; the score and
+// value MMAs come from two threads, so the value MMAs of a tile go out as
+// soon as its probabilities are ready (releasing ring slots early) while
+// score MMAs keep the pipe busy; and the ring moves in chunk pairs, so a tile
+// costs the score thread three waits and one commit and the value thread one
+// wait and two commits.
 //
 //   warp 0      TMA producer: q~ once, then the latents in 64-column chunks
-//               (6 KB: 48 keys x 64 d_c) through the ring
+//               (KT keys x 64 d_c) through the ring
 //   warp 1      TMEM owner; issues the score MMAs (one thread)
 //   warps 2..5  softmax, one head per TMEM lane; lazy rescale of acc^T when a
 //               head's running max grows by more than 2^8; partial-state store
@@ -49,23 +54,25 @@
 // of the P^T buffer that follows q~: they only feed S rows 96..127, which
 // nothing reads.
 //
-// TMEM columns: S buffers at 0 and 64 (48 columns each), acc^T blocks at
+// TMEM columns: S buffers at 0 and 64 (KT columns each), acc^T blocks at
 // 128 + 96*blk.
 #include "internal.h"
 #include "ptx.cuh"
+#include "ws_layout.h"
 
 namespace gmla {
 namespace latent_tc {
 
 constexpr int HMAX = 96;
-constexpr int KT = 48;                    // keys per tile: N of the score product
+constexpr int KT = kLatentTileKeys;       // keys per tile (48 or 64): N of the score product
+static_assert(KT == 48 || KT == 64, "tile keys");
 constexpr int NUM_THREADS = 224;
 constexpr int NCHUNK = 8;                 // 64-wide d_c chunks per tile (d_c <= 512)
 constexpr int QCHUNK = HMAX * 128;        // 12 KB: one d_c chunk of q~ for 96 heads
 constexpr int Q_BYTES = NCHUNK * QCHUNK;  // 96 KB
-constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row (48 keys used) per head
-constexpr int CCHUNK = KT * 128;          // 6 KB: one d_c chunk of a 48-key tile
-constexpr int NSLOT = 18;                 // latent ring depth in chunks
+constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row (up to 64 keys) per head
+constexpr int CCHUNK = KT * 128;          // one d_c chunk of a tile: KT keys x 64 d_c (6 or 8 KB)
+constexpr int NSLOT = KT == 64 ? 14 : 18; // latent ring depth in chunks (1.75 or 2.25 tiles)
 constexpr int NPAIR = NSLOT / 2;          // the ring moves in chunk pairs (one 128-row d_c block)
 constexpr int NPT = NCHUNK / 2;           // chunk pairs per tile
 constexpr int NEARLY_PAIRS = 3;           // score chunk pairs of tile j issued before the value MMAs of tile j-1
@@ -78,10 +85,15 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-pat
 
 // Ring reuse: the chunks move in pairs (2i, 2i+1) -- the two halves of d_c
 // block i -- through NPAIR pair slots.  Pair q of tile j sits in pair slot
-// (4j + q) % NPAIR; its previous user belongs to tile j-2 or earlier, whose
-// value MMAs were issued an iteration before the score MMAs that need the
-// slot.  The two chunks of a pair are adjacent, so one MN-major descriptor
-// with a chunk-sized leading offset spans the 128-row d_c block.
+// (4j + q) % NPAIR, so its previous user is pair 4j + q - NPAIR: with 9 pair
+// slots (48-key tiles) a pair of tile j-2 or j-3; with 7 (64-key tiles) pair
+// q+1 of tile j-2 for q < 3 and pair 0 of tile j-1 for q = 3.  The early pairs
+// (0..2) of tile j therefore wait only on tiles j-2 and before, whose value
+// MMAs went out while the score MMAs of tile j-1 ran, and a late pair on a
+// release of tile j-1 that needs nothing of tile j.  No wait is on a later
+// tile, so the ring cannot deadlock.  The two chunks of a pair are adjacent,
+// so one MN-major descriptor with a chunk-sized leading offset spans the
+// 128-row d_c block.
 //
 // Barriers are per tile (rotating over NTB tiles), not per slot, so that a
 // tile costs the MMA thread two data waits (pairs 0..2, pair 3) and two
@@ -91,7 +103,7 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-pat
 // release of tile j-2 or j-3, by which time the MMA thread has consumed
 // tile j-NTB; the producer waits for the release of tile j-2 or j-3 only
 // after it observed the releases of tiles j-4 and earlier.
-static_assert(NSLOT % 2 == 0 && NPAIR >= 2 * NPT + 1, "ring depth");
+static_assert(NSLOT % 2 == 0 && NPAIR >= NPT + NEARLY_PAIRS, "early pairs of tile j reuse slots of tile j-2");
 static_assert(P_BYTES >= 32 * 128, "P^T buffer must cover the q~ tail");
 
 struct Params {
@@ -129,6 +141,29 @@ __device__ __forceinline__ void tmem_ld48(uint32_t taddr, float *v) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 48; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 64 consecutive float32 columns of this thread's TMEM lane (warp-wide).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *v) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]),
+        "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]),
+        "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr), "r"(taddr + 32)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // OR of `v` over the `count` threads of named barrier `id` (all of them must call).
@@ -333,7 +368,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (got) {
         tc_fence_after();
         if (active) {
-          tmem_ld48(tmem + lane_off + TM_S + sb * 64, x);
+          if constexpr (KT == 64)
+            tmem_ld64(tmem + lane_off + TM_S + sb * 64, x);
+          else
+            tmem_ld48(tmem + lane_off + TM_S + sb * 64, x);
         } else {
 #pragma unroll
           for (int c = 0; c < KT; ++c) x[c] = -INFINITY;

@@ -175,14 +175,14 @@ static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T
                                         int64_t d_c, const gmla_bf16 *W_k, const gmla_bf16 *W_v, gmla_bf16 *Q,
                                         gmla_bf16 *G, gmla_bf16 *C, int64_t cache_len_max, int64_t cache_pos,
                                         gmla_bf16 *K, gmla_bf16 *V, gmla_stream_t stream) {
-  if (!X || B <= 0 || T <= 0 || d_model <= 0 || d_c <= 0) return GMLA_ERR_ARG;
+  if (!X || B <= 0 || T <= 0 || d_model <= 0) return GMLA_ERR_ARG;
   if ((Q && !W_q) || (G && !W_g) || (C && !W_c) || (K && !W_k) || (V && !W_v)) return GMLA_ERR_ARG;
   if ((K || V) && !C) return GMLA_ERR_ARG;
-  if (C && (cache_pos < 0 || cache_len_max <= 0 || cache_pos + T > cache_len_max)) return GMLA_ERR_ARG;
+  if (C && (d_c <= 0 || cache_pos < 0 || cache_len_max <= 0 || cache_pos + T > cache_len_max)) return GMLA_ERR_ARG;
   const void *ptrs[] = {X, W_q, W_g, W_c, W_k, W_v, Q, G, C, K, V};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return GMLA_ERR_ARG;
-  if (d_model % 128 != 0 || d_c % 64 != 0) return GMLA_ERR_UNSUPPORTED;
+  if (d_model % 128 != 0 || (C && d_c % 64 != 0)) return GMLA_ERR_UNSUPPORTED;
   if (h0 < 0 || h1 <= h0 || h1 > d_model / 128) return GMLA_ERR_ARG;
   if (B * T > 0x7fffffffLL || cache_len_max > 0x7fffffffLL || B > 65535) return GMLA_ERR_UNSUPPORTED;
   unsigned *st = status_ptr();

@@ -15,6 +15,7 @@ namespace gmla {
 
 constexpr size_t kWsAlign = 256;
 constexpr size_t kTensorMapBytes = 128;  // sizeof(CUtensorMap)
+constexpr int kLatentTileKeys = 48;      // keys per tile of the latent decode kernel (48 or 64)
 
 inline size_t ws_round(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
 

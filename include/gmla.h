@@ -106,7 +106,8 @@ typedef void *gmla_stream_t; /* a cudaStream_t */
  *          cache_pos + T <= cache_len_max.  Required when K or V is requested.
  *  K, V    [B, T, d_model] outputs, may be NULL.  They are expanded from the
  *          bfloat16 latents just written to C.
- * Needs no scratch memory.
+ * d_c and the cache arguments matter only when C is given.  Needs no
+ * scratch memory.
  * Returns GMLA_ERR_ARG for null required pointers, cache_pos + T >
  * cache_len_max or misalignment; GMLA_ERR_UNSUPPORTED when d_model is not a
  * multiple of 128 or d_c not a multiple of 64.

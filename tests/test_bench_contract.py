@@ -64,6 +64,11 @@ def test_workload_arithmetic():
     assert latents == pytest.approx(4.295e9, rel=1e-3)
     extra = b.decode_bytes(32, 131072) - latents
     assert 0 < extra < 0.02 * latents  # W_k, W_v, q, G and O on top of the cache
+    # decode over explicit K, V at the softmax page's shape: Q, K, V, O = 394.0 MB
+    assert b.plain_decode_bytes() == 2 * 8 * 96 * 128 * (2 * 1001 + 2)
+    assert b.plain_decode_bytes() == pytest.approx(393.8e6, rel=1e-3)
+    # full layer prefill: a1 5.05e12 + a2 2.06e11 + a3 8.248e11 + a5 2.474e12 = 8.556e12 flop
+    assert b.layer_flops() == pytest.approx(8.556e12, rel=1e-3)
     # the sweep's lengths are the cost table's, whose dot-product orders they reproduce
     assert b.SWEEP_T == (8192, 131072, 1048576)
     for t, order in zip(b.SWEEP_T, b.SWEEP_PAGE["dot_products_per_head"]):

@@ -32,16 +32,16 @@ int main() {
   for (auto &c : cases) {
     const long long B = c[0], L = c[1], H = c[2], dc = c[3];
     int S, kps;
-    latent_plan(B, L, 48, &S, &kps);
+    latent_plan(B, L, kLatentTileKeys, &S, &kps);
     for (int per_seq = 0; per_seq < 2; ++per_seq) {
       const size_t need = latent_layout_bytes(B, H, dc, S, per_seq);
       for (unsigned long long k = 0; k < 16; ++k) {
         const unsigned long long base = 0x7f0000000000ull + 16 * k;
         const LatentLayout o = latent_layout(base, B, H, dc, S, per_seq);
         std::printf("%s{\"kind\":\"decode\",\"B\":%lld,\"L\":%lld,\"H\":%lld,\"dc\":%lld,\"S\":%d,\"kps\":%d,"
-                    "\"per_seq\":%d,\"base\":%llu,\"need\":%zu,\"qt\":%zu,\"pm\":%zu,\"pl\":%zu,\"pacc\":%zu,"
+                    "\"tile\":%d,\"per_seq\":%d,\"base\":%llu,\"need\":%zu,\"qt\":%zu,\"pm\":%zu,\"pl\":%zu,\"pacc\":%zu,"
                     "\"lse2\":%zu,\"maps\":%zu,\"lens\":%zu,\"end\":%zu}",
-                    first ? "" : ",", B, L, H, dc, S, kps, per_seq, base, need, o.qt, o.pm, o.pl, o.pacc, o.lse2,
+                    first ? "" : ",", B, L, H, dc, S, kps, kLatentTileKeys, per_seq, base, need, o.qt, o.pm, o.pl, o.pacc, o.lse2,
                     o.maps, o.lens, o.end);
         first = false;
       }
@@ -104,7 +104,7 @@ def test_split_plan_covers_every_key_once(layouts):
         if r["kind"] != "decode":
             continue
         S, kps, L = r["S"], r["kps"], r["L"]
-        assert kps % 48 == 0 and S >= 1
+        assert kps % r["tile"] == 0 and S >= 1
         assert (S - 1) * kps < L <= S * kps, r   # no empty split, nothing left over
 
 
