@@ -9,11 +9,13 @@
 //   absorb   q~[b,h,:] = scale * log2(e) * W_k^(h)T q_h, stored as bfloat16
 //   stream   tensor-core split-KV pass over the latents (attn_latent_tc.cu):
 //            per split the running max m, sum l and acc[h,:] = sum_s p_s c_s
-//   combine  exact log-sum-exp merge of the splits, c^ = acc / l, then
-//            o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store -- or, for
-//            the partial form over a key range, the merged state itself
-//            (c^ and its log-sum-exp), which gmla_decode_combine later merges
-//            with the states of other key ranges.
+//   merge    exact log-sum-exp merge of the splits, c^ = acc / l (the
+//            partial form over a key range stops here: c^ and its
+//            log-sum-exp, which gmla_decode_combine later merges with the
+//            states of other key ranges)
+//   W_v      o_h = W_v^(h) c^_h, gate sigmoid(G), bfloat16 store.
+// gmla_decode_combine, which has no scratch for c^, does the last two in one
+// kernel (combine_kernel).
 #include <math.h>
 
 #include <mutex>
@@ -49,11 +51,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ---------------------------------------------------------------- absorb
-// grid (H, ceil(d_c / 128), ceil(B / AB)), 128 threads: thread j owns latent
-// column c = 128*y + j for the AB sequences b0 .. b0+AB-1.  The CTA first
-// copies its 128 x 128 tile of W_k^(h) and the AB query rows of head h into
-// shared memory with 16-byte loads that are all in flight at once, then
-// forms the products from shared memory.
+// grid (H, ceil(d_c / 128), ceil(B / AB)), 128 threads.  The CTA copies its
+// 128 x 128 tile of W_k^(h) (rows d, columns 128*y ..) and the AB query rows
+// of head h into shared memory with 16-byte loads that are all in flight at
+// once.  Thread t then owns four adjacent columns c = 128*y + 4*(t % 32) and
+// eight sequences b = b0 + 8*(t / 32) ..: per four rows d it reads four
+// 8-byte groups of W_k (adjacent lanes, adjacent addresses) and eight float4
+// of q (the same address across the warp: a broadcast) for 128 multiply-adds.
 constexpr int AB = 32;
 constexpr size_t kAbsorbSmem = AB * HD * sizeof(float) + HD * 128 * sizeof(uint16_t);  // 48 KB
 
@@ -71,52 +75,70 @@ __global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict_
       *reinterpret_cast<uint4 *>(ws + d * 128 + 8 * v) =
           *reinterpret_cast<const uint4 *>(Wk + ((size_t)h * HD + d) * dc + c0 + 8 * v);
   }
-  for (int i = threadIdx.x; i < nb * 16; i += 128) {
+  for (int i = threadIdx.x; i < AB * 16; i += 128) {
     const int j = i >> 4, v = i & 15;
-    const uint4 u = *reinterpret_cast<const uint4 *>(Q + (size_t)(b0 + j) * H * HD + (size_t)h * HD + 8 * v);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     float *dst = qs + j * HD + 8 * v;
+    if (j < nb) {
+      const uint4 u = *reinterpret_cast<const uint4 *>(Q + (size_t)(b0 + j) * H * HD + (size_t)h * HD + 8 * v);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      dst[2 * e] = __uint_as_float(w[e] << 16);
-      dst[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      for (int e = 0; e < 4; ++e) {
+        dst[2 * e] = __uint_as_float(w[e] << 16);
+        dst[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dst[e] = 0.f;  // rows past B: computed, never stored
     }
   }
   __syncthreads();
-  const int c = threadIdx.x;
-  if (c >= ncol) return;
-  float acc[AB];
+  const int cq = 4 * (threadIdx.x & 31);  // first of this thread's four columns
+  const int jg = 8 * (threadIdx.x >> 5);  // first of its eight sequences
+  if (cq >= ncol) return;
+  float acc[8][4];
 #pragma unroll
-  for (int j = 0; j < AB; ++j) acc[j] = 0.f;
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
 #pragma unroll 2
   for (int d = 0; d < HD; d += 4) {
-    float w[4];
+    float w[4][4];  // [row d+e][column cq+k]
 #pragma unroll
-    for (int e = 0; e < 4; ++e) w[e] = bf16_to_f32(ws[(d + e) * 128 + c]);
+    for (int e = 0; e < 4; ++e) {
+      const uint2 u = *reinterpret_cast<const uint2 *>(ws + (d + e) * 128 + cq);
+      w[e][0] = __uint_as_float(u.x << 16);
+      w[e][1] = __uint_as_float(u.x & 0xFFFF0000u);
+      w[e][2] = __uint_as_float(u.y << 16);
+      w[e][3] = __uint_as_float(u.y & 0xFFFF0000u);
+    }
 #pragma unroll
-    for (int j = 0; j < AB; ++j) {
-      if (j < nb) {
-        const float4 q4 = *reinterpret_cast<const float4 *>(qs + j * HD + d);
-        acc[j] = fmaf(q4.x, w[0], acc[j]);
-        acc[j] = fmaf(q4.y, w[1], acc[j]);
-        acc[j] = fmaf(q4.z, w[2], acc[j]);
-        acc[j] = fmaf(q4.w, w[3], acc[j]);
-      }
+    for (int j = 0; j < 8; ++j) {
+      const float4 q4 = *reinterpret_cast<const float4 *>(qs + (jg + j) * HD + d);
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[j][k] = fmaf(qv[e], w[e][k], acc[j][k]);
     }
   }
 #pragma unroll
-  for (int j = 0; j < AB; ++j)
-    if (j < nb) qt[((size_t)(b0 + j) * H + h) * dc + c0 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j] * sl2));
+  for (int j = 0; j < 8; ++j) {
+    if (jg + j < nb) {
+      uint2 o;
+      o.x = pack_bf16x2(acc[j][0] * sl2, acc[j][1] * sl2);
+      o.y = pack_bf16x2(acc[j][2] * sl2, acc[j][3] * sl2);
+      *reinterpret_cast<uint2 *>(qt + ((size_t)(b0 + jg + j) * H + h) * dc + c0 + cq) = o;
+    }
+  }
 }
 
-// ---------------------------------------------------------------- combine
-// grid (H, ceil(B / CB)), CT threads.  Phase 1: warp bb computes the weights
-// 2^(m_s - M) / sum_s l_s 2^(m_s - M) of the S partial states of sequence
-// b0 + bb (lanes over s).  Phase 2: c^ = sum_s w_s acc_s over all (sequence,
-// column) pairs, 16-byte loads with eight states in flight per thread.
-// Phase 3 (full form): o_h = W_v^(h) c^, two threads per output row (one half
-// of d_c each), then the gate and the bfloat16 store.  The partial form
-// stores c^ and the merged log-sum-exp instead.
+// ---------------------------------------------------------------- combine (gmla_decode_combine)
+// Merge of n states and W_v in one kernel, for gmla_decode_combine, which has
+// no scratch for c^.  grid (H, ceil(B / CB)), CT threads.  Phase 1: warp bb
+// computes the weights 2^(m_s - M) / sum_s l_s 2^(m_s - M) of the states of
+// sequence b0 + bb (lanes over s).  Phase 2: c^ = sum_s w_s acc_s over all
+// (sequence, column) pairs into shared memory.  Phase 3: o_h = W_v^(h) c^ with
+// W_v read in whole rows, then the gate and the bfloat16 store.
 constexpr int CB = 8;
 constexpr int CT = 256;
 static_assert(CT / 32 == CB, "one warp per sequence in phase 1");
@@ -128,11 +150,9 @@ struct CombineParams {
   int n_splits, B, H, dc;
   const uint16_t *Wv, *G;
   uint16_t *O;
-  float *lse2;                   // full form: [B,H] log2-domain log-sum-exp (for the debug weights), may be null
-  float *out_lse, *out_chat;     // partial form: [B,H] natural-log log-sum-exp, [B,H,dc] c^
+  float *lse2;  // [B,H] log2-domain log-sum-exp, may be null
 };
 
-template <bool kPartial>
 __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
   extern __shared__ __align__(16) float csm[];  // chat [CB][dc] | split weights [CB][n_splits]
   const int h = blockIdx.x, b0 = blockIdx.y * CB;
@@ -159,13 +179,7 @@ __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     __syncwarp();
     for (int s = lane; s < S; s += 32) wsp[warp * S + s] *= inv;
-    if (lane == 0) {
-      const float l2 = Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY;
-      if (kPartial)
-        P.out_lse[(size_t)b * P.H + h] = l2 * kLn2;
-      else if (P.lse2)
-        P.lse2[(size_t)b * P.H + h] = l2;
-    }
+    if (lane == 0 && P.lse2) P.lse2[(size_t)b * P.H + h] = Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY;
   }
   __syncthreads();
   {
@@ -192,47 +206,235 @@ __global__ void __launch_bounds__(CT) combine_kernel(const CombineParams P) {
           a.w = fmaf(ws, v[u].w, a.w);
         }
       }
-      if (kPartial)
-        *reinterpret_cast<float4 *>(P.out_chat + ((size_t)(b0 + bb) * P.H + h) * dc + c) = a;
-      else
-        *reinterpret_cast<float4 *>(chat + bb * dc + c) = a;
+      *reinterpret_cast<float4 *>(chat + bb * dc + c) = a;
     }
   }
-  if (kPartial) return;
   __syncthreads();
-  const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
-  const int c_lo = half * (dc / 2), c_hi = c_lo + dc / 2;
-  const uint16_t *w = P.Wv + ((size_t)h * HD + r) * dc;
-  float o[CB];
+  // o_h[b, r] = sum_c W_v[h*128 + r, c] c^[b, c].  Warp w owns rows
+  // 64*(w >> 2) .. +63 and sequences bp, bp+1 (bp = 2*(w & 3)); lane l owns the
+  // columns 16l .. 16l+15 (d_c <= 512) of every row, so a warp reads whole rows
+  // of W_v (coalesced) and keeps its columns of c^ in registers.  Per block of
+  // 32 rows each lane holds 32 partial sums per sequence; a transpose-reduce
+  // across the warp (31 shuffles) leaves lane l with the full sum of row l.
+  const int bp = 2 * (warp & 3), rbase = 64 * (warp >> 2);
+  const int c0 = 16 * lane;
+  const bool cols_ok = c0 < dc;
+  float cx[2][16];
 #pragma unroll
-  for (int bb = 0; bb < CB; ++bb) o[bb] = 0.f;
-#pragma unroll 4
-  for (int c = c_lo; c < c_hi; c += 8) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(w + c);
-    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+  for (int k = 0; k < 2; ++k)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float w0 = __uint_as_float(ww[e] << 16), w1 = __uint_as_float(ww[e] & 0xFFFF0000u);
+    for (int e = 0; e < 16; ++e) cx[k][e] = (cols_ok && bp + k < nb) ? chat[(bp + k) * dc + c0 + e] : 0.f;
+#pragma unroll 1
+  for (int rb = 0; rb < 64; rb += 32) {
+    float part[2][32];
 #pragma unroll
-      for (int bb = 0; bb < CB; ++bb) {
-        if (bb < nb) {
-          o[bb] = fmaf(w0, chat[bb * dc + c + 2 * e], o[bb]);
-          o[bb] = fmaf(w1, chat[bb * dc + c + 2 * e + 1], o[bb]);
+    for (int i = 0; i < 32; ++i) {
+      float w[16];
+      if (cols_ok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(P.Wv + ((size_t)h * HD + rbase + rb + i) * dc + c0);
+        const uint4 v0 = src[0], v1 = src[1];
+        const uint32_t ww[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          w[2 * e] = __uint_as_float(ww[e] << 16);
+          w[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
         }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) a = fmaf(w[e], cx[k][e], a);
+        part[k][i] = a;
       }
     }
-  }
+    // transpose-reduce: after the step with offset o each lane keeps the half
+    // of its rows whose index has lane's bit o, adding its partner's copy
 #pragma unroll
-  for (int bb = 0; bb < CB; ++bb) o[bb] += __shfl_xor_sync(0xffffffffu, o[bb], 1);
-  if (half == 0) {
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool up = (lane & o) != 0;
 #pragma unroll
-    for (int bb = 0; bb < CB; ++bb) {
-      if (bb < nb) {
-        const size_t oi = (size_t)(b0 + bb) * P.H * HD + (size_t)h * HD + r;
-        float v = o[bb];
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+          const float send = up ? part[k][i] : part[k][i + o];
+          const float keep = up ? part[k][i + o] : part[k][i];
+          part[k][i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (bp + k < nb) {
+        const size_t oi = (size_t)(b0 + bp + k) * P.H * HD + (size_t)h * HD + rbase + rb + lane;
+        float v = part[k][0];
         if (P.G) v *= sigmoidf_(bf16_to_f32(P.G[oi]));
         P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- merge (decode path)
+// The exact log-sum-exp merge of the S split states, one thread per float4 of
+// the [B*H, d_c] state: thread i reads its four columns of every split (all
+// loads in flight), the S maxima and sums of its (b, h) row (shared by the
+// d_c/4 threads of the row: served from L1), and writes c^ = sum_s w_s acc_s
+// -- in place over split 0 (each thread reads its own slot before writing it)
+// or into the caller's buffer (partial form), with the row's log-sum-exp.
+struct MergeParams {
+  const float *part_m, *part_l;  // [S, BH]; part_l null: every sum is 1
+  const float *part_acc;         // [S, BH, dc]
+  float *chat;                   // [BH, dc]
+  float m_scale;                 // to log2 units
+  int S, BH, dc;
+  float *lse2;                   // [BH] log2 domain, or null
+  float *lse_nat;                // [BH] natural log, or null
+};
+
+constexpr int MT = 256;
+
+__global__ void __launch_bounds__(MT) merge_kernel(const MergeParams P) {
+  const int per_row = P.dc / 4;
+  const size_t i4 = blockIdx.x * (size_t)MT + threadIdx.x;
+  if (i4 >= (size_t)P.BH * per_row) return;
+  const size_t bh = i4 / per_row;
+  const int S = P.S;
+  float M = -INFINITY;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, P.part_m[(size_t)s * P.BH + bh] * P.m_scale);
+  const float4 *src = reinterpret_cast<const float4 *>(P.part_acc) + i4;
+  const size_t split4 = (size_t)P.BH * per_row;
+  float Lsum = 0.f;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < S; s0 += 8) {
+    float e[8];
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      const float m = s < S ? P.part_m[(size_t)s * P.BH + bh] * P.m_scale : -INFINITY;
+      e[u] = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
+      // an empty state (weight 0) left no acc: never read it
+      v[u] = e[u] != 0.f ? src[(size_t)s * split4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      if (s < S) Lsum += (P.part_l ? P.part_l[(size_t)s * P.BH + bh] : 1.f) * e[u];
+      a.x = fmaf(e[u], v[u].x, a.x);
+      a.y = fmaf(e[u], v[u].y, a.y);
+      a.z = fmaf(e[u], v[u].z, a.z);
+      a.w = fmaf(e[u], v[u].w, a.w);
+    }
+  }
+  // no visible key in any state: c^ = 0, log-sum-exp -inf
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  reinterpret_cast<float4 *>(P.chat)[i4] = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+  if (i4 % per_row == 0) {
+    const float l2 = Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY;
+    if (P.lse2) P.lse2[bh] = l2;
+    if (P.lse_nat) P.lse_nat[bh] = l2 * kLn2;
+  }
+}
+
+// ---------------------------------------------------------------- W_v and gate (decode path)
+// o_h[b, r] = sum_c W_v[h*128 + r, c] c^[b, h, c], then the gate.  grid (H,
+// ceil(B / CB)), 256 threads.  W_v^(h) (128 rows of d_c, contiguous) streams
+// through shared memory in chunks of 32 rows by 1-D bulk copies, two chunks in
+// flight; c^ of the CTA's CB sequences is staged in shared memory once.  For
+// each chunk, warp w takes sequence b0 + w with lanes over columns (lane l:
+// columns 16l .. 16l+15, read as two 16-byte words per row, conflict-free) and
+// holds 32 partial sums; a transpose-reduce across the warp (31 shuffles)
+// leaves lane l with the full sum of the chunk's row l.
+struct WvParams {
+  const float *chat;  // [B, H, dc]
+  const uint16_t *Wv, *G;
+  uint16_t *O;
+  int B, H, dc;
+  unsigned *status;
+};
+
+constexpr int WV_ROWS = 32;  // rows of W_v per chunk
+
+__global__ void __launch_bounds__(CT) wv_kernel(const WvParams P) {
+  extern __shared__ __align__(128) uint8_t wv_sm[];
+  const int dc = P.dc;
+  const uint32_t chunk_bytes = WV_ROWS * dc * 2;
+  uint16_t *wbuf = reinterpret_cast<uint16_t *>(wv_sm);                  // [2][WV_ROWS][dc]
+  float *csm = reinterpret_cast<float *>(wv_sm + 2 * chunk_bytes);       // [CB][dc]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(csm + CB * dc);           // [2]
+  const int h = blockIdx.x, b0 = blockIdx.y * CB;
+  const int nb = min(CB, P.B - b0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NCHUNK = HD / WV_ROWS;
+  const uint16_t *wsrc = P.Wv + (size_t)h * HD * dc;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_barrier_init();
+    for (int c = 0; c < 2; ++c) {
+      mbar_arrive_expect_tx(&bar[c], chunk_bytes);
+      bulk_load(wbuf + (size_t)c * WV_ROWS * dc, wsrc + (size_t)c * WV_ROWS * dc, chunk_bytes, &bar[c]);
+    }
+  }
+  for (int i4 = threadIdx.x; i4 < nb * dc / 4; i4 += CT) {
+    const int bb = (i4 * 4) / dc, c = (i4 * 4) % dc;
+    *reinterpret_cast<float4 *>(csm + bb * dc + c) =
+        *reinterpret_cast<const float4 *>(P.chat + ((size_t)(b0 + bb) * P.H + h) * dc + c);
+  }
+  __syncthreads();  // c^ staged; barrier initialisation visible
+  const int c0 = 16 * lane;
+  const bool cols_ok = c0 < dc;
+  const bool seq_ok = warp < nb;
+  float cx[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) cx[e] = (cols_ok && seq_ok) ? csm[warp * dc + c0 + e] : 0.f;
+  bool ok = true;
+#pragma unroll 1
+  for (int ch = 0; ch < NCHUNK; ++ch) {
+    const int buf = ch & 1;
+    ok = ok && mbar_wait(&bar[buf], (ch >> 1) & 1, P.status);
+    const uint16_t *wch = wbuf + (size_t)buf * WV_ROWS * dc;
+    float part[WV_ROWS];
+#pragma unroll
+    for (int i = 0; i < WV_ROWS; ++i) {
+      float a = 0.f;
+      if (cols_ok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(wch + (size_t)i * dc + c0);
+        const uint4 v0 = src[0], v1 = src[1];
+        const uint32_t ww[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          a = fmaf(__uint_as_float(ww[e] << 16), cx[2 * e], a);
+          a = fmaf(__uint_as_float(ww[e] & 0xFFFF0000u), cx[2 * e + 1], a);
+        }
+      }
+      part[i] = a;
+    }
+    __syncthreads();  // every warp has read this chunk: its buffer may be refilled
+    if (threadIdx.x == 0 && ok && ch + 2 < NCHUNK) {
+      mbar_arrive_expect_tx(&bar[buf], chunk_bytes);
+      bulk_load(wbuf + (size_t)buf * WV_ROWS * dc, wsrc + (size_t)(ch + 2) * WV_ROWS * dc, chunk_bytes, &bar[buf]);
+    }
+    // transpose-reduce: after the step with offset o each lane keeps the half
+    // of its rows whose index has lane's bit o, adding its partner's copy
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < o; ++i) {
+        const float send = up ? part[i] : part[i + o];
+        const float keep = up ? part[i + o] : part[i];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    if (seq_ok && ok) {
+      const size_t oi = (size_t)(b0 + warp) * P.H * HD + (size_t)h * HD + ch * WV_ROWS + lane;
+      float v = part[0];
+      if (P.G) v *= sigmoidf_(bf16_to_f32(P.G[oi]));
+      P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
   }
 }
@@ -336,27 +538,38 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
       return -1;
   }
   {
-    CombineParams P;
-    P.part_m = pm;
-    P.part_l = pl;
-    P.part_acc = pacc;
-    P.m_scale = 1.f;
-    P.n_splits = S;
-    P.B = a.B;
-    P.H = a.H;
-    P.dc = a.dc;
-    P.Wv = a.Wv;
-    P.G = a.G;
-    P.O = a.O;
-    P.lse2 = lse2;
-    P.out_lse = a.out_lse;
-    P.out_chat = a.out_chat;
-    const dim3 grid(a.H, (a.B + CB - 1) / CB);
-    const size_t shm = sizeof(float) * (CB * a.dc + CB * S);
-    if (a.out_chat)
-      combine_kernel<true><<<grid, CT, shm, stream>>>(P);
-    else
-      combine_kernel<false><<<grid, CT, shm, stream>>>(P);
+    // merge the split states: in place over split 0 of the partial accumulators,
+    // or into the caller's buffers for the partial form
+    MergeParams M;
+    M.part_m = pm;
+    M.part_l = pl;
+    M.part_acc = pacc;
+    M.chat = a.out_chat ? a.out_chat : pacc;
+    M.m_scale = 1.f;
+    M.S = S;
+    M.BH = a.B * a.H;
+    M.dc = a.dc;
+    M.lse2 = a.out_chat ? nullptr : lse2;
+    M.lse_nat = a.out_lse;
+    const size_t n4 = (size_t)M.BH * a.dc / 4;
+    merge_kernel<<<(unsigned)((n4 + MT - 1) / MT), MT, 0, stream>>>(M);
+  }
+  if (!a.out_chat) {
+    WvParams W;
+    W.chat = pacc;
+    W.Wv = a.Wv;
+    W.G = a.G;
+    W.O = a.O;
+    W.B = a.B;
+    W.H = a.H;
+    W.dc = a.dc;
+    W.status = a.status;
+    const size_t shm = 2 * (size_t)WV_ROWS * a.dc * 2 + sizeof(float) * CB * a.dc + 2 * sizeof(uint64_t);
+    if (!set_smem_limit_once(reinterpret_cast<const void *>(wv_kernel), (int)(2 * WV_ROWS * 512 * 2 +
+                                                                               sizeof(float) * CB * 512 + 16),
+                             kSmemWv))
+      return -1;
+    wv_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), CT, shm, stream>>>(W);
   }
   if (a.weights && a.lens)
     weights_fix_varlen_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, lens_dev, a.H, a.B * a.H,
@@ -395,9 +608,7 @@ int launch_latent_combine(const float *lse, const float *chat, int n, int B, int
   P.G = G;
   P.O = O;
   P.lse2 = nullptr;
-  P.out_lse = nullptr;
-  P.out_chat = nullptr;
-  combine_kernel<false><<<dim3(H, (B + CB - 1) / CB), CT, sizeof(float) * (CB * dc + CB * n), stream>>>(P);
+  combine_kernel<<<dim3(H, (B + CB - 1) / CB), CT, sizeof(float) * (CB * dc + CB * n), stream>>>(P);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

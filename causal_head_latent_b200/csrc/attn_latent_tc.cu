@@ -72,7 +72,8 @@ constexpr int QCHUNK = HMAX * 128;        // 12 KB: one d_c chunk of q~ for 96 h
 constexpr int Q_BYTES = NCHUNK * QCHUNK;  // 96 KB
 constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row (up to 64 keys) per head
 constexpr int CCHUNK = KT * 128;          // one d_c chunk of a tile: KT keys x 64 d_c (6 or 8 KB)
-constexpr int NSLOT = KT == 64 ? 14 : 18; // latent ring depth in chunks (1.75 or 2.25 tiles)
+constexpr int PBUF = 1;                   // P^T buffers (2: the softmax of tile j waits for tile j-2's value MMAs)
+constexpr int NSLOT = KT == 64 ? 14 : (PBUF == 2 ? 16 : 18);  // latent ring depth in chunks
 constexpr int NPAIR = NSLOT / 2;          // the ring moves in chunk pairs (one 128-row d_c block)
 constexpr int NPT = NCHUNK / 2;           // chunk pairs per tile
 constexpr int NEARLY_PAIRS = 3;           // score chunk pairs of tile j issued before the value MMAs of tile j-1
@@ -105,6 +106,7 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-pat
 // after it observed the releases of tiles j-4 and earlier.
 static_assert(NSLOT % 2 == 0 && NPAIR >= NPT + NEARLY_PAIRS, "early pairs of tile j reuse slots of tile j-2");
 static_assert(P_BYTES >= 32 * 128, "P^T buffer must cover the q~ tail");
+static_assert(PBUF == 1 || (PBUF == 2 && KT == 48), "a second P^T buffer fits next to the 48-key ring only");
 
 struct Params {
   const uint16_t *C;  // latent cache [B, Lmax, dc] (for the L2 prefetch stream)
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sq = base;
   uint8_t *sp = sq + Q_BYTES;  // directly after q~: it holds the padded rows' tail
-  uint8_t *sc = sp + P_BYTES;  // Q_BYTES + P_BYTES is a multiple of 1024
+  uint8_t *sc = sp + PBUF * P_BYTES;  // Q_BYTES + P_BYTES is a multiple of 1024
   float *alpha_s = reinterpret_cast<float *>(sc + NSLOT * CCHUNK);
   uint64_t *bars = reinterpret_cast<uint64_t *>(alpha_s + 128);
   uint64_t *bar_q = bars;
@@ -340,7 +342,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int ks = 0; ks < KT / 16; ++ks)
             umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
-                         sdesc_sw128(ap + ks * 32, 16, 1024), idPV, (j > 0 || ks > 0) ? 1u : 0u);
+                         sdesc_sw128(ap + (j % PBUF) * P_BYTES + ks * 32, 16, 1024), idPV,
+                         (j > 0 || ks > 0) ? 1u : 0u);
           // rel[.][1] also tells the softmax of tile j+1 that P^T and acc^T are free
           if (blk & 1) umma_commit(&rel[2 * (j % NTB) + (blk >> 1)]);
         }
@@ -393,10 +396,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (k0 + c < k_end) wrow[k0 + c] = x[c];
       }
       const bool need = head_ok && mx > m_used + kRescaleThreshold;
-      // P^T and acc^T are free once the value MMAs of tile j-1 have completed
+      // P^T buffer j % PBUF is free once the value MMAs of tile j - PBUF have completed
       bool ready = got;
-      if (got && j >= 1) {
-        const int jp = j - 1;
+      if (got && j >= PBUF) {
+        const int jp = j - PBUF;
         ready = __all_sync(0xffffffffu, mbar_wait(&rel[2 * (jp % NTB) + 1], (jp / NTB) & 1, p.status));
         tc_fence_after();
       }
@@ -404,6 +407,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (bar_or(1, 128, !ready)) {  // a wait gave up: every softmax thread leaves together
           ok = false;
           break;
+        }
+        if (PBUF > 1 && j >= 1) {
+          // the rescale below touches acc^T: the value MMAs of tile j-1 must have completed
+          const int jp = j - 1;
+          const bool r1 = __all_sync(0xffffffffu, mbar_wait(&rel[2 * (jp % NTB) + 1], (jp / NTB) & 1, p.status));
+          if (bar_or(1, 128, !r1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
         }
         float alpha = 1.f;
         if (need) {
@@ -441,11 +454,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         pk[c / 2] = pack_bf16x2(p0, p1);
       }
       l += rs;
-      // P^T row h (free: the value MMAs of tile j-1 have completed)
+      // P^T row h of buffer j % PBUF (free: the value MMAs of tile j - PBUF have completed)
       if (active) {
 #pragma unroll
         for (int u = 0; u < KT / 8; ++u)
-          *reinterpret_cast<uint4 *>(prow + ((u ^ sw) << 4)) =
+          *reinterpret_cast<uint4 *>(prow + (j % PBUF) * P_BYTES + ((u ^ sw) << 4)) =
               make_uint4(pk[u * 4 + 0], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
       }
       fence_proxy_async_smem();
@@ -493,7 +506,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 size_t smem_bytes() {
-  return 1024 + Q_BYTES + P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 4 * NTB + 9) + 16;
+  return 1024 + Q_BYTES + PBUF * P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 4 * NTB + 9) + 16;
 }
 
 }  // namespace latent_tc

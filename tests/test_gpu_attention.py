@@ -54,6 +54,25 @@ def test_prefill_matches_oracle(g, B, H, Tq, Tk, causal):
     assert np.abs(w - wref).max() < 1e-4
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_many_items_per_cta(g, causal):
+    """More query pairs than SMs (B=2, H=40, T=1100: 400 items), so running CTAs
+    take over the items of CTAs that have not started and carry their
+    pipelines from one item to the next; the last pair of every head has rows
+    for its first query tile only.  Every output and log-sum-exp is compared."""
+    B, H, T = 2, 40, 1100
+    inp = prefill_qkv(171 + causal, B, T, H, gate=True)
+    Q, K, V, G = (to_dev(inp[k]) for k in ("Q", "K", "V", "G"))
+    O = torch.empty_like(Q)
+    L = torch.empty(B, H, T, device="cuda")
+    g.gmla_attend_prefill(Q, K, V, O, causal=causal, G=G, lse=L)
+    g.gmla_get_device_status()
+    ref, lref = orc.attention(inp["Q"], inp["K"], inp["V"], causal=causal, want_lse=True)
+    ref = orc.gate(ref.reshape(B, T, -1), inp["G"]).reshape(ref.shape)
+    assert_parity(f64(O), ref, "O over 400 items")
+    np.testing.assert_allclose(f64(L), lref, rtol=0, atol=2e-4)
+
+
 def test_prefill_gate_and_layout(g):
     inp = prefill_qkv(7, 2, 260, 3, gate=True)
     O, _, _ = run_prefill(g, inp, gate=True)
