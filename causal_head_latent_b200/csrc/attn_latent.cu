@@ -69,11 +69,20 @@ __global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict_
   const int h = blockIdx.x, c0 = blockIdx.y * 128, b0 = blockIdx.z * AB;
   const int nb = min(AB, B - b0);
   const int ncol = min(128, dc - c0);  // 64 or 128 (d_c is a multiple of 64)
-  for (int i = threadIdx.x; i < HD * 16; i += 128) {
-    const int d = i >> 4, v = i & 15;
-    if (8 * v < ncol)
-      *reinterpret_cast<uint4 *>(ws + d * 128 + 8 * v) =
-          *reinterpret_cast<const uint4 *>(Wk + ((size_t)h * HD + d) * dc + c0 + 8 * v);
+  {
+    // sixteen 16-byte loads per thread, all issued before the first store
+    uint4 t[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = threadIdx.x + 128 * k, d = i >> 4, v = i & 15;
+      t[k] = 8 * v < ncol ? *reinterpret_cast<const uint4 *>(Wk + ((size_t)h * HD + d) * dc + c0 + 8 * v)
+                          : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = threadIdx.x + 128 * k, d = i >> 4, v = i & 15;
+      *reinterpret_cast<uint4 *>(ws + d * 128 + 8 * v) = t[k];
+    }
   }
   for (int i = threadIdx.x; i < AB * 16; i += 128) {
     const int j = i >> 4, v = i & 15;
@@ -341,13 +350,14 @@ __global__ void __launch_bounds__(MT) merge_kernel(const MergeParams P) {
 
 // ---------------------------------------------------------------- W_v and gate (decode path)
 // o_h[b, r] = sum_c W_v[h*128 + r, c] c^[b, h, c], then the gate.  grid (H,
-// ceil(B / CB)), 256 threads.  W_v^(h) (128 rows of d_c, contiguous) streams
-// through shared memory in chunks of 32 rows by 1-D bulk copies, two chunks in
-// flight; c^ of the CTA's CB sequences is staged in shared memory once.  For
-// each chunk, warp w takes sequence b0 + w with lanes over columns (lane l:
+// ceil(B / WV_CB)), 256 threads.  W_v^(h) (128 rows of d_c, contiguous)
+// streams through shared memory in chunks of 32 rows by 1-D bulk copies, two
+// chunks in flight; c^ of the CTA's WV_CB = 16 sequences is staged in shared
+// memory once (each head's W_v is read by ceil(B / 16) CTAs).  For each chunk,
+// warp w takes sequences b0 + 2w, b0 + 2w + 1 with lanes over columns (lane l:
 // columns 16l .. 16l+15, read as two 16-byte words per row, conflict-free) and
-// holds 32 partial sums; a transpose-reduce across the warp (31 shuffles)
-// leaves lane l with the full sum of the chunk's row l.
+// holds 32 partial sums per sequence; a transpose-reduce across the warp (31
+// shuffles per sequence) leaves lane l with the full sums of the chunk's row l.
 struct WvParams {
   const float *chat;  // [B, H, dc]
   const uint16_t *Wv, *G;
@@ -357,16 +367,17 @@ struct WvParams {
 };
 
 constexpr int WV_ROWS = 32;  // rows of W_v per chunk
+constexpr int WV_CB = 16;    // sequences per CTA (two per warp)
 
 __global__ void __launch_bounds__(CT) wv_kernel(const WvParams P) {
   extern __shared__ __align__(128) uint8_t wv_sm[];
   const int dc = P.dc;
   const uint32_t chunk_bytes = WV_ROWS * dc * 2;
   uint16_t *wbuf = reinterpret_cast<uint16_t *>(wv_sm);                  // [2][WV_ROWS][dc]
-  float *csm = reinterpret_cast<float *>(wv_sm + 2 * chunk_bytes);       // [CB][dc]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(csm + CB * dc);           // [2]
-  const int h = blockIdx.x, b0 = blockIdx.y * CB;
-  const int nb = min(CB, P.B - b0);
+  float *csm = reinterpret_cast<float *>(wv_sm + 2 * chunk_bytes);       // [WV_CB][dc]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(csm + WV_CB * dc);        // [2]
+  const int h = blockIdx.x, b0 = blockIdx.y * WV_CB;
+  const int nb = min(WV_CB, P.B - b0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NCHUNK = HD / WV_ROWS;
   const uint16_t *wsrc = P.Wv + (size_t)h * HD * dc;
@@ -379,39 +390,54 @@ __global__ void __launch_bounds__(CT) wv_kernel(const WvParams P) {
       bulk_load(wbuf + (size_t)c * WV_ROWS * dc, wsrc + (size_t)c * WV_ROWS * dc, chunk_bytes, &bar[c]);
     }
   }
-  for (int i4 = threadIdx.x; i4 < nb * dc / 4; i4 += CT) {
-    const int bb = (i4 * 4) / dc, c = (i4 * 4) % dc;
-    *reinterpret_cast<float4 *>(csm + bb * dc + c) =
-        *reinterpret_cast<const float4 *>(P.chat + ((size_t)(b0 + bb) * P.H + h) * dc + c);
+  // c^ of the CTA's sequences: up to eight 16-byte loads per thread, all in flight
+  for (int base = 0; base < nb * dc / 4; base += 8 * CT) {
+    float4 t[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i4 = base + threadIdx.x + k * CT;
+      const int bb = (i4 * 4) / dc, c = (i4 * 4) % dc;
+      t[k] = i4 < nb * dc / 4 ? *reinterpret_cast<const float4 *>(P.chat + ((size_t)(b0 + bb) * P.H + h) * dc + c)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i4 = base + threadIdx.x + k * CT;
+      if (i4 < nb * dc / 4) *reinterpret_cast<float4 *>(csm + i4 * 4) = t[k];
+    }
   }
   __syncthreads();  // c^ staged; barrier initialisation visible
   const int c0 = 16 * lane;
   const bool cols_ok = c0 < dc;
-  const bool seq_ok = warp < nb;
-  float cx[16];
+  const int bw = 2 * warp;  // this warp's first sequence within the CTA
+  float cx[2][16];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) cx[e] = (cols_ok && seq_ok) ? csm[warp * dc + c0 + e] : 0.f;
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) cx[k][e] = (cols_ok && bw + k < nb) ? csm[(bw + k) * dc + c0 + e] : 0.f;
   bool ok = true;
 #pragma unroll 1
   for (int ch = 0; ch < NCHUNK; ++ch) {
     const int buf = ch & 1;
     ok = ok && mbar_wait(&bar[buf], (ch >> 1) & 1, P.status);
     const uint16_t *wch = wbuf + (size_t)buf * WV_ROWS * dc;
-    float part[WV_ROWS];
+    float part[2][WV_ROWS];
 #pragma unroll
     for (int i = 0; i < WV_ROWS; ++i) {
-      float a = 0.f;
+      float a0 = 0.f, a1 = 0.f;
       if (cols_ok) {
         const uint4 *src = reinterpret_cast<const uint4 *>(wch + (size_t)i * dc + c0);
         const uint4 v0 = src[0], v1 = src[1];
         const uint32_t ww[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          a = fmaf(__uint_as_float(ww[e] << 16), cx[2 * e], a);
-          a = fmaf(__uint_as_float(ww[e] & 0xFFFF0000u), cx[2 * e + 1], a);
+          const float w0 = __uint_as_float(ww[e] << 16), w1 = __uint_as_float(ww[e] & 0xFFFF0000u);
+          a0 = fmaf(w1, cx[0][2 * e + 1], fmaf(w0, cx[0][2 * e], a0));
+          a1 = fmaf(w1, cx[1][2 * e + 1], fmaf(w0, cx[1][2 * e], a1));
         }
       }
-      part[i] = a;
+      part[0][i] = a0;
+      part[1][i] = a1;
     }
     __syncthreads();  // every warp has read this chunk: its buffer may be refilled
     if (threadIdx.x == 0 && ok && ch + 2 < NCHUNK) {
@@ -424,17 +450,22 @@ __global__ void __launch_bounds__(CT) wv_kernel(const WvParams P) {
     for (int o = 16; o >= 1; o >>= 1) {
       const bool up = (lane & o) != 0;
 #pragma unroll
-      for (int i = 0; i < o; ++i) {
-        const float send = up ? part[i] : part[i + o];
-        const float keep = up ? part[i + o] : part[i];
-        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+          const float send = up ? part[k][i] : part[k][i + o];
+          const float keep = up ? part[k][i + o] : part[k][i];
+          part[k][i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
     }
-    if (seq_ok && ok) {
-      const size_t oi = (size_t)(b0 + warp) * P.H * HD + (size_t)h * HD + ch * WV_ROWS + lane;
-      float v = part[0];
-      if (P.G) v *= sigmoidf_(bf16_to_f32(P.G[oi]));
-      P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (bw + k < nb && ok) {
+        const size_t oi = (size_t)(b0 + bw + k) * P.H * HD + (size_t)h * HD + ch * WV_ROWS + lane;
+        float v = part[k][0];
+        if (P.G) v *= sigmoidf_(bf16_to_f32(P.G[oi]));
+        P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+      }
     }
   }
 }
@@ -564,12 +595,11 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     W.H = a.H;
     W.dc = a.dc;
     W.status = a.status;
-    const size_t shm = 2 * (size_t)WV_ROWS * a.dc * 2 + sizeof(float) * CB * a.dc + 2 * sizeof(uint64_t);
-    if (!set_smem_limit_once(reinterpret_cast<const void *>(wv_kernel), (int)(2 * WV_ROWS * 512 * 2 +
-                                                                               sizeof(float) * CB * 512 + 16),
-                             kSmemWv))
+    const size_t shm = 2 * (size_t)WV_ROWS * a.dc * 2 + sizeof(float) * WV_CB * a.dc + 2 * sizeof(uint64_t);
+    if (!set_smem_limit_once(reinterpret_cast<const void *>(wv_kernel),
+                             (int)(2 * WV_ROWS * 512 * 2 + sizeof(float) * WV_CB * 512 + 16), kSmemWv))
       return -1;
-    wv_kernel<<<dim3(a.H, (a.B + CB - 1) / CB), CT, shm, stream>>>(W);
+    wv_kernel<<<dim3(a.H, (a.B + WV_CB - 1) / WV_CB), CT, shm, stream>>>(W);
   }
   if (a.weights && a.lens)
     weights_fix_varlen_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, lens_dev, a.H, a.B * a.H,
