@@ -30,7 +30,7 @@ namespace gmla {
 int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
                      int k_base, int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l,
                      float *part_acc, float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens,
-                     unsigned *status, cudaStream_t stream);
+                     const LatentItem *items, int n_items, unsigned *status, cudaStream_t stream);
 int latent_tc_tile_keys();
 
 namespace latent {
@@ -301,6 +301,11 @@ struct MergeParams {
   int S, BH, dc;
   float *lse2;                   // [BH] log2 domain, or null
   float *lse_nat;                // [BH] natural log, or null
+  // Work-item records (null: S splits per sequence in [S, BH] order): the
+  // states of sequence b are records b and seq_off[b] .. seq_off[b+1]-1 of
+  // [R, H] (and [R, H, dc]); H heads per sequence.
+  const int *seq_off;
+  int H;
 };
 
 constexpr int MT = 256;
@@ -310,11 +315,23 @@ __global__ void __launch_bounds__(MT) merge_kernel(const MergeParams P) {
   const size_t i4 = blockIdx.x * (size_t)MT + threadIdx.x;
   if (i4 >= (size_t)P.BH * per_row) return;
   const size_t bh = i4 / per_row;
-  const int S = P.S;
+  const int col4 = (int)(i4 % per_row);
+  // record of state s of this (b, h)
+  int S = P.S;
+  size_t b_seq = 0, h = bh, x0 = 0;
+  if (P.seq_off) {
+    b_seq = bh / P.H;
+    h = bh % P.H;
+    x0 = (size_t)P.seq_off[b_seq];
+    S = 1 + (P.seq_off[b_seq + 1] - P.seq_off[b_seq]);
+  }
+  auto rec = [&](int st) -> size_t {
+    if (!P.seq_off) return (size_t)st * P.BH + bh;
+    return (st == 0 ? b_seq : x0 + st - 1) * (size_t)P.H + h;
+  };
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, P.part_m[(size_t)s * P.BH + bh] * P.m_scale);
-  const float4 *src = reinterpret_cast<const float4 *>(P.part_acc) + i4;
-  const size_t split4 = (size_t)P.BH * per_row;
+  for (int st = 0; st < S; ++st) M = fmaxf(M, P.part_m[rec(st)] * P.m_scale);
+  const float4 *src = reinterpret_cast<const float4 *>(P.part_acc);
   float Lsum = 0.f;
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s0 = 0; s0 < S; s0 += 8) {
@@ -322,16 +339,17 @@ __global__ void __launch_bounds__(MT) merge_kernel(const MergeParams P) {
     float4 v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int s = s0 + u;
-      const float m = s < S ? P.part_m[(size_t)s * P.BH + bh] * P.m_scale : -INFINITY;
+      const int st = s0 + u;
+      const size_t r = st < S ? rec(st) : 0;
+      const float m = st < S ? P.part_m[r] * P.m_scale : -INFINITY;
       e[u] = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
       // an empty state (weight 0) left no acc: never read it
-      v[u] = e[u] != 0.f ? src[(size_t)s * split4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[u] = e[u] != 0.f ? src[r * per_row + col4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int s = s0 + u;
-      if (s < S) Lsum += (P.part_l ? P.part_l[(size_t)s * P.BH + bh] : 1.f) * e[u];
+      const int st = s0 + u;
+      if (st < S) Lsum += (P.part_l ? P.part_l[rec(st)] : 1.f) * e[u];
       a.x = fmaf(e[u], v[u].x, a.x);
       a.y = fmaf(e[u], v[u].y, a.y);
       a.z = fmaf(e[u], v[u].z, a.z);
@@ -505,48 +523,65 @@ void latent_plan(long long B, long long L, int *n_splits, int *keys_per_split) {
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc) {
   int S, kps;
   latent_plan(B, L, &S, &kps);
-  return latent_layout_bytes(B, H, dc, S, false);
+  return latent_layout_bytes(B, H, dc, (long long)S * B, false);
 }
 
-// With per-sequence lengths the plan follows cache_len_max, and the workspace
-// also holds one 128-byte tensor map and one int32 length per sequence.
+// With per-sequence lengths the workspace holds the states of up to
+// latent_varlen_records(B, cache_len_max) work items, and per sequence a
+// 128-byte tensor map, an int32 length and a record offset.
 size_t latent_varlen_workspace_bytes(long long B, long long cache_len_max, long long H, long long dc) {
-  int S, kps;
-  latent_plan(B, cache_len_max, &S, &kps);
-  return latent_layout_bytes(B, H, dc, S, true);
+  return latent_layout_bytes(B, H, dc, latent_varlen_records(B, cache_len_max, latent_tc_tile_keys()), true);
 }
 
-// The three launches for a given split plan (S splits of kps keys over the
-// key range [a.k0, a.L), or [0, lens[b]) per sequence) and workspace.
+// The launches for a given split plan (S splits of kps keys over the key
+// range [a.k0, a.L)) and workspace; with per-sequence lengths (a.lens) the
+// plan is the work-item plan of those lengths and S, kps are not used.
 static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaStream_t stream) {
   using namespace latent;
   static_assert(sizeof(CUtensorMap) == kTensorMapBytes, "tensor map size");
+  static_assert(sizeof(LatentItem) == 16, "work item size");
   uint8_t *base = static_cast<uint8_t *>(a.workspace);
-  const LatentLayout lay = latent_layout(reinterpret_cast<uintptr_t>(base), a.B, a.H, a.dc, S, a.lens != nullptr);
+  const long long records =
+      a.lens ? latent_varlen_records(a.B, a.cache_len_max, latent_tc_tile_keys()) : (long long)S * a.B;
+  const LatentLayout lay = latent_layout(reinterpret_cast<uintptr_t>(base), a.B, a.H, a.dc, records, a.lens != nullptr);
   uint16_t *qt = reinterpret_cast<uint16_t *>(base + lay.qt);
   float *pm = reinterpret_cast<float *>(base + lay.pm);
   float *pl = reinterpret_cast<float *>(base + lay.pl);
   float *pacc = reinterpret_cast<float *>(base + lay.pacc);
   float *lse2 = reinterpret_cast<float *>(base + lay.lse2);
   CUtensorMap *maps = nullptr;
-  int *lens_dev = nullptr;
+  int *lens_dev = nullptr, *offs_dev = nullptr;
+  LatentItem *items_dev = nullptr;
+  long long n_items = 0;
   if (a.lens) {
-    // per-sequence 2-D latent maps (d_c, lens[b]) and lengths, copied before the launches;
-    // the map region starts on a 256-byte boundary (TMA reads maps at 64-byte alignment)
+    // per-sequence 2-D latent maps (d_c, lens[b]), lengths, work items and record
+    // offsets, copied before the launches; the map region starts on a 256-byte
+    // boundary (TMA reads maps at 64-byte alignment)
     maps = reinterpret_cast<CUtensorMap *>(base + lay.maps);
     lens_dev = reinterpret_cast<int *>(base + lay.lens);
+    items_dev = reinterpret_cast<LatentItem *>(base + lay.items);
+    offs_dev = reinterpret_cast<int *>(base + lay.offs);
     std::vector<CUtensorMap> hm((size_t)a.B);
-    std::vector<int> hl((size_t)a.B);
+    std::vector<int> hl((size_t)a.B), ho((size_t)a.B + 1);
     for (int b = 0; b < a.B; ++b) {
       const long long dims[2] = {a.dc, a.lens[b]}, strides[1] = {a.dc};
       const unsigned box[2] = {64, (unsigned)latent_tc_tile_keys()};
       if (!make_tmap_bf16(&hm[b], a.C + (size_t)b * a.cache_len_max * a.dc, 2, dims, strides, box)) return -1;
       hl[b] = (int)a.lens[b];
     }
+    int kps_v = 0;
+    n_items = latent_varlen_plan(a.lens, a.B, latent_tc_tile_keys(), records, &kps_v, nullptr, nullptr);
+    if (n_items < 1 || n_items > records) return -1;
+    std::vector<LatentItem> hi((size_t)n_items);
+    latent_varlen_plan(a.lens, a.B, latent_tc_tile_keys(), records, &kps_v, hi.data(), ho.data());
+    S = 1;
     // pageable sources: the copies are staged before cudaMemcpyAsync returns
     if (cudaMemcpyAsync(maps, hm.data(), hm.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice, stream) !=
             cudaSuccess ||
-        cudaMemcpyAsync(lens_dev, hl.data(), hl.size() * sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        cudaMemcpyAsync(lens_dev, hl.data(), hl.size() * sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(items_dev, hi.data(), hi.size() * sizeof(LatentItem), cudaMemcpyHostToDevice, stream) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(offs_dev, ho.data(), ho.size() * sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess)
       return -1;
   }
 
@@ -565,7 +600,7 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     if (!make_tmap_bf16(&tc, a.C, 3, dcm, scm, bc)) return -1;
     const int w_ld = a.lens ? (int)a.cache_len_max : a.L;
     if (launch_latent_tc(tq, tc, a.C, a.cache_len_max, a.B, a.L, (int)a.k0, a.H, a.dc, S, kps, pm, pl, pacc,
-                         a.weights, w_ld, maps, lens_dev, a.status, stream) != 0)
+                         a.weights, w_ld, maps, lens_dev, items_dev, (int)n_items, a.status, stream) != 0)
       return -1;
   }
   {
@@ -582,6 +617,8 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     M.dc = a.dc;
     M.lse2 = a.out_chat ? nullptr : lse2;
     M.lse_nat = a.out_lse;
+    M.seq_off = offs_dev;
+    M.H = a.H;
     const size_t n4 = (size_t)M.BH * a.dc / 4;
     merge_kernel<<<(unsigned)((n4 + MT - 1) / MT), MT, 0, stream>>>(M);
   }
@@ -692,7 +729,9 @@ int launch_attend_latent_noalloc(const LatentArgs &args, cudaStream_t stream) {
   latent_plan(args.B, args.L, &S, &kps);
   // fewer splits when the default plan's partial states do not fit (the array
   // is 256-byte aligned, so the layout starts at its first byte)
-  auto fits = [&](int s) { return latent_layout(0, args.B, args.H, args.dc, s, false).end <= kNoAllocScratchBytes; };
+  auto fits = [&](int s) {
+    return latent_layout(0, args.B, args.H, args.dc, (long long)s * args.B, false).end <= kNoAllocScratchBytes;
+  };
   while (S > 1 && !fits(S)) --S;
   if (!fits(S)) return -3;
   const int KT = latent_tc_tile_keys();

@@ -121,6 +121,10 @@ struct Params {
   // whose row extent makes a ragged last tile read zeros past lens[b].
   const CUtensorMap *tmC_seq;
   const int *lens;
+  // Work items (null: blockIdx = b * n_splits + split): this CTA streams rows
+  // [items[i].y, items[i].z) of sequence items[i].x into record items[i].w of
+  // the [R, H] partial states.
+  const int4 *items;
   unsigned *status;
 };
 
@@ -205,15 +209,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_idle + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int b = blockIdx.x / p.n_splits;
-  const int split = blockIdx.x % p.n_splits;
-  const int Lb = p.lens ? p.lens[b] : p.L;
-  const int k_begin = p.k_base + split * p.keys_per_split;
-  const int k_end = min(Lb, k_begin + p.keys_per_split);
+  int b, k_begin, k_end;
+  size_t rec;  // first of this CTA's H partial-state records
+  if (p.items) {
+    const int4 it = p.items[blockIdx.x];
+    b = it.x;
+    k_begin = it.y;
+    k_end = it.z;
+    rec = (size_t)it.w * p.H;
+  } else {
+    b = blockIdx.x / p.n_splits;
+    const int split = blockIdx.x % p.n_splits;
+    const int Lb = p.lens ? p.lens[b] : p.L;
+    k_begin = p.k_base + split * p.keys_per_split;
+    k_end = min(Lb, k_begin + p.keys_per_split);
+    rec = ((size_t)split * p.B + b) * p.H;
+  }
   if (k_end <= k_begin) {
     // A split past the end of a shorter sequence: an empty partial state,
     // which the combine skips.  The whole CTA leaves before any barrier.
-    const size_t rec = ((size_t)split * p.B + b) * p.H;
     for (int h = threadIdx.x; h < p.H; h += NUM_THREADS) {
       p.part_m[rec + h] = -INFINITY;
       p.part_l[rec + h] = 0.f;
@@ -472,7 +486,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool fin = !bar_or(1, 128, !mbar_wait(acc_done, 0, p.status));
       if (fin) {
         tc_fence_after();
-        const size_t rec = ((size_t)split * p.B + b) * p.H;
         if (head_ok) {
           p.part_m[rec + h] = m_used;
           p.part_l[rec + h] = l;
@@ -516,7 +529,7 @@ int latent_tc_tile_keys() { return latent_tc::KT; }
 int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint16_t *C, long long Lmax, int B, int L,
                      int k_base, int H, int dc, int n_splits, int keys_per_split, float *part_m, float *part_l,
                      float *part_acc, float *weights, int w_ld, const CUtensorMap *tmC_seq, const int *lens,
-                     unsigned *status, cudaStream_t stream) {
+                     const LatentItem *items, int n_items, unsigned *status, cudaStream_t stream) {
   using namespace latent_tc;
   auto kern = latent_decode_kernel;
   const size_t smem = smem_bytes();
@@ -538,8 +551,11 @@ int launch_latent_tc(const CUtensorMap &tmQt, const CUtensorMap &tmC, const uint
   p.w_ld = w_ld;
   p.tmC_seq = tmC_seq;
   p.lens = lens;
+  p.items = reinterpret_cast<const int4 *>(items);
   p.status = status;
-  kern<<<B * n_splits, NUM_THREADS, smem, stream>>>(tmQt, tmC, p);
+  const long long grid = items ? (long long)n_items : (long long)B * n_splits;
+  if (grid < 1 || grid > 0x7fffffffLL) return -1;
+  kern<<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tmQt, tmC, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
