@@ -8,9 +8,16 @@
 //   warp 0      TMA producer, 4-stage ring (A 16 KB + B 32 KB per stage)
 //   warp 1      TMEM owner and MMA issuer: per chunk 4 x tcgen05.mma
 //               (M=128, N=256, K=16), both operands K-major
-//   warps 2..5  epilogue: TMEM -> registers -> bf16 -> global, one output
-//               row per thread; two TMEM accumulators (2 x 256 columns) let
-//               the epilogue of tile i overlap the main loop of tile i+1.
+//   warps 2..5  epilogue: TMEM -> registers -> bf16, one output row per
+//               thread; two TMEM accumulators (2 x 256 columns) let the
+//               epilogue of tile i overlap the main loop of tile i+1.  Each
+//               warp stages its 32 rows x 64 columns in shared memory (two
+//               4 KB buffers, 128-byte swizzle) and one lane writes them out
+//               with a TMA bulk store, so the store of one chunk overlaps the
+//               conversion of the next and the writes leave as whole lines.
+//               Boxes that would cross an output batch or the end of the rows
+//               (and outputs whose layout TMA cannot address) are written by
+//               per-thread 16-byte stores instead.
 // The tile order walks groups of 16 m-tiles across all n-tiles so the CTAs
 // resident at one time share A rows and B columns in L2.
 #include "internal.h"
@@ -25,9 +32,13 @@ constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int NUM_THREADS = 192;
 constexpr int GROUP_M = 16;
 
+constexpr int OUT_ROWS = 32, OUT_COLS = 64;          // one epilogue warp's store box
+constexpr int OUT_BYTES = OUT_ROWS * OUT_COLS * 2;    // 4 KB
+
 struct Smem {
   uint8_t a[STAGES][A_BYTES];
   uint8_t b[STAGES][B_BYTES];
+  uint8_t out[4][2][OUT_BYTES];  // per epilogue warp, double-buffered
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t acc_full[2];
@@ -44,6 +55,7 @@ struct Params {
   int n_tiles_total;
   int total_tiles;
   int k_chunks;
+  int tma_out[3];     // problem i is written through tmO_i (3-D map: N, rows_per_b, batches; box 64 x 32 x 1)
 };
 
 struct TileCoord {
@@ -73,7 +85,8 @@ __device__ __forceinline__ TileCoord tile_coord(const Params &P, int idx) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
-                const Params P) {
+                const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
+                const __grid_constant__ CUtensorMap tmO2, const Params P) {
   extern __shared__ uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -150,6 +163,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    uint32_t staged = 0;  // boxes this warp has handed to TMA (buffer rotation)
     int it = 0;
     for (int idx = blockIdx.x; idx < P.total_tiles; idx += gridDim.x, ++it) {
       const TileCoord tc = tile_coord(P, idx);
@@ -157,29 +171,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&sm.acc_full[ab], (it >> 1) & 1, status)) break;
       tc_fence_after();
       const GemmOut &o = P.g.prob[tc.prob];
+      const CUtensorMap *mo = tc.prob == 0 ? &tmO0 : (tc.prob == 1 ? &tmO1 : &tmO2);
       const int bidx = tc.mt / P.m_tiles_per_b;
       const int t = (tc.mt % P.m_tiles_per_b) * BM + r;
       const bool row_ok = t < P.g.a_rows;
       const long long m = (long long)bidx * P.g.a_rows + t;
       uint16_t *orow = o.out + (m / o.rows_per_b) * o.sb + (m % o.rows_per_b) * o.st + o.off;
+      // this warp's 32 rows as one box: all inside the problem's rows and inside one output batch
+      const int t_box = t - lane;
+      const long long m_box = m - lane;
+      const bool boxed = P.tma_out[tc.prob] && t_box + OUT_ROWS <= P.g.a_rows &&
+                         m_box % o.rows_per_b + OUT_ROWS <= o.rows_per_b;
       const uint32_t tD = tmem + ab * BN + lane_off;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tD + c * 32, v);
-        const int n0 = tc.nt * BN + c * 32;
-        if (row_ok && n0 < o.N) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + n0);
+      for (int c = 0; c < BN / OUT_COLS; ++c) {
+        float v[OUT_COLS];
+        tmem_ld32(tD + c * OUT_COLS, *reinterpret_cast<float(*)[32]>(v));
+        tmem_ld32(tD + c * OUT_COLS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        const int n0 = tc.nt * BN + c * OUT_COLS;
+        if (n0 >= o.N) continue;
+        if (boxed) {
+          uint8_t *buf = sm.out[quarter][staged & 1];
+          if (staged >= 2) {
+            if (lane == 0) bulk_wait_group_read<1>();  // the store that used this buffer has read it
+            __syncwarp();
+          }
+          // row `lane` of the box: 16-byte chunk q at position q ^ (row % 8) (128-byte swizzle)
+          uint4 *dst = reinterpret_cast<uint4 *>(buf + lane * 128);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]), pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
-                                pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]), pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]));
+          for (int q = 0; q < 8; ++q)
+            dst[q ^ (lane & 7)] =
+                make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]), pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
+                           pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]), pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(mo, buf, n0, (int)(m_box % o.rows_per_b), (int)(m_box / o.rows_per_b));
+            bulk_commit_group();
+          }
+          ++staged;
+        } else if (row_ok) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (n0 + 32 * h >= o.N) break;
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + n0 + 32 * h);
+            const float *w = v + 32 * h;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(w[q * 8 + 0], w[q * 8 + 1]), pack_bf16x2(w[q * 8 + 2], w[q * 8 + 3]),
+                                  pack_bf16x2(w[q * 8 + 4], w[q * 8 + 5]), pack_bf16x2(w[q * 8 + 6], w[q * 8 + 7]));
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
     }
+    if (lane == 0) bulk_wait_group<0>();  // the bulk stores have finished before the CTA exits
+    __syncwarp();
   }
 
   __syncwarp();  // lane 0 of the producer / MMA warps ran its loop alone
@@ -207,10 +256,30 @@ int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &
   P.total_tiles = P.m_tiles * P.n_tiles_total;
   P.k_chunks = (a.K + BK - 1) / BK;
   if (P.total_tiles <= 0 || P.k_chunks <= 0) return 0;
+  // Output maps: problem i is stored by TMA when its rows can be described as
+  // a 3-D tiled map (16-byte aligned base and row / batch strides).
+  CUtensorMap tmO[3];
+  const long long rows_total = (long long)a.a_rows * a.a_batches;
+  for (int i = 0; i < 3; ++i) {
+    P.tma_out[i] = 0;
+    if (i >= a.n_problems) continue;
+    const GemmOut &o = a.prob[i];
+    const uint16_t *base = o.out + o.off;
+    const long long nb = (rows_total + o.rows_per_b - 1) / o.rows_per_b;
+    const long long sb = nb > 1 ? o.sb : o.rows_per_b * o.st;
+    const bool addressable = (reinterpret_cast<uintptr_t>(base) & 15) == 0 && o.st % 8 == 0 && sb % 8 == 0 &&
+                             o.st >= o.N && sb >= o.rows_per_b * o.st && o.N > 0;
+    if (!addressable) continue;
+    const long long dims[3] = {o.N, o.rows_per_b, nb}, strides[2] = {o.st, sb};
+    const unsigned box[3] = {OUT_COLS, OUT_ROWS, 1};
+    P.tma_out[i] = make_tmap_bf16(&tmO[i], base, 3, dims, strides, box) ? 1 : 0;
+  }
+  for (int i = 0; i < 3; ++i)
+    if (!P.tma_out[i]) tmO[i] = tmA;  // never read: the kernel stores problem i directly
   const int grid = P.total_tiles < num_sms() ? P.total_tiles : num_sms();
   const CUtensorMap &b1 = a.n_problems > 1 ? tmB[1] : tmB[0];
   const CUtensorMap &b2 = a.n_problems > 2 ? tmB[2] : tmB[0];
-  gemm_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB[0], b1, b2, P);
+  gemm_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB[0], b1, b2, tmO[0], tmO[1], tmO[2], P);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
