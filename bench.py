@@ -102,9 +102,10 @@ PROFILED_TRAFFIC = {
                             "bytes": 604.206080e6 + 184.497408e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192); profiles/attn_prefill_kernel__causal_B1_H96_T8192.md"},
-    "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu"], "sha1": "6e0d1461be5365d74184699ffca2b97f62e4f5c3",
-                           "bytes": (542.555648e6 - 536.870912e6 + 8 * 536.870912e6) + 29.40288e6 + 13.388032e6
-                                    + 56.862208e6 + 19.710976e6,
+    "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu"],
+                           "sha1": "72f7f1208e551bc6d4dae6d8f1c93687b871a222",
+                           "bytes": (543.941888e6 - 536.870912e6 + 8 * 536.870912e6) + 29.335808e6 + 13.388032e6
+                                    + 56.872192e6 + 19.710720e6,
                            "how": "ncu dram bytes of the four kernels of one call at L=16384 (absorb, stream, merge, "
                                   "W_v); the stream kernel's cache reads (B*L*1 KB) scaled x8 to L=131072, the rest "
                                   "(q~, partial states, W_k, W_v) unscaled; profiles/gmla_attend_decode__B32_L16384.md"},
