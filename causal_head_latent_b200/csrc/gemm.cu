@@ -239,6 +239,165 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+
+// ------------------------------------------------------------------ split-K for few rows
+// With at most 32 output rows (a decode step: one new token per sequence) a
+// launch of 128 x 256 tiles has fewer tiles than SMs (W_o at d_model = 12288:
+// 48), and each CTA is capped by its own TMA ingress while the others idle.
+// Here a cluster of sk CTAs shares one tile, each taking a contiguous 1/sk of
+// the K chunks; CTAs 1 .. sk-1 stage their float32 partial rows in their own
+// shared memory and send them to CTA 0 with one bulk copy each, and CTA 0 adds
+// them to its accumulator and writes the bf16 tile.  Only TMEM lanes 0..31
+// (the rows) carry data, so one epilogue warp per CTA does the work.
+constexpr int SK_MAX = 2;
+constexpr int SK_STAGES = 4;
+constexpr int SK_ROWS = 32;
+constexpr int SK_PART_BYTES = SK_ROWS * BN * 4;  // 32 KB: one CTA's float32 partial rows
+
+struct SmemSK {
+  uint8_t a[SK_STAGES][A_BYTES];
+  uint8_t b[SK_STAGES][B_BYTES];
+  uint8_t part[SK_MAX - 1][SK_PART_BYTES];  // CTA 0: partials received; others: slot 0 stages their own
+  uint64_t full[SK_STAGES];
+  uint64_t empty[SK_STAGES];
+  uint64_t acc_full;
+  uint64_t recv;  // CTA 0: the partials of CTAs 1 .. SK-1 have landed
+  uint32_t tmem_base;
+};
+constexpr size_t kSmemBytesSK = sizeof(SmemSK) + 1024;
+
+// 16-byte chunk q (of 64) of row r of a partial, swizzled so that a warp
+// whose lanes hold consecutive rows touches all banks.
+__device__ __forceinline__ uint32_t sk_off(int r, int q) { return r * (BN * 4) + ((q ^ (r & 7)) << 4); }
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                       const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                       const Params P, const int sk) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemSK &sm = *reinterpret_cast<SmemSK *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  unsigned *status = P.g.status;
+  const int rank = (int)cluster_ctarank();
+  const int tile = blockIdx.x / sk;
+  const int kc0 = (int)((long long)P.k_chunks * rank / sk), kc1 = (int)((long long)P.k_chunks * (rank + 1) / sk);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SK_STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.recv, 1);
+    if (rank == 0) mbar_arrive_expect_tx(&sm.recv, (uint32_t)(sk - 1) * SK_PART_BYTES);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of every CTA initialised (CTA 0's receive barrier armed)
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const TileCoord tc = tile_coord(P, tile);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const CUtensorMap *mb = tc.prob == 0 ? &tmB0 : (tc.prob == 1 ? &tmB1 : &tmB2);
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(mb);
+      for (int kc = kc0, g = 0; kc < kc1; ++kc, ++g) {
+        const int s = g % SK_STAGES;
+        if (!mbar_wait(&sm.empty[s], ((g / SK_STAGES) & 1) ^ 1, status)) break;
+        mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
+        tma_load_3d(sm.a[s], &tmA, &sm.full[s], kc * BK, P.g.a_row0, 0);
+        tma_load_2d(sm.b[s], mb, &sm.full[s], kc * BK, tc.nt * BN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
+      bool ok = true;
+      for (int kc = kc0, g = 0; kc < kc1; ++kc, ++g) {
+        const int s = g % SK_STAGES;
+        if (!(ok = mbar_wait(&sm.full[s], (g / SK_STAGES) & 1, status))) break;
+        tc_fence_after();
+        const uint32_t aa = smem_u32(sm.a[s]), bb = smem_u32(sm.b[s]);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16_ss(tmem, sdesc_sw128(aa + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 32, 16, 1024), idesc,
+                       (kc > kc0 || kk > 0) ? 1u : 0u);
+        umma_commit(&sm.empty[s]);
+      }
+      if (ok) umma_commit(&sm.acc_full);
+    }
+  } else if ((warp & 3) == 0) {
+    // the epilogue warp of TMEM lanes 0..31: row `lane` of the tile
+    const bool got = mbar_wait(&sm.acc_full, 0, status);
+    tc_fence_after();
+    if (rank != 0) {
+      // stage this CTA's partial rows and send them to CTA 0
+      uint8_t *stage = sm.part[0];
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + c * 32, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float4 *>(stage + sk_off(lane, c * 8 + q)) =
+              got ? make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t dst = mapa_shared(smem_u32(sm.part[rank - 1]), 0);
+        bulk_copy_to_peer(dst, stage, SK_PART_BYTES, mapa_shared(smem_u32(&sm.recv), 0));
+      }
+    } else {
+      const bool have = mbar_wait(&sm.recv, 0, status) && got;
+      const GemmOut &o = P.g.prob[tc.prob];
+      const int t = lane;  // row
+      const bool row_ok = have && t < P.g.a_rows;
+      uint16_t *orow = o.out + (t / o.rows_per_b) * o.sb + (t % o.rows_per_b) * o.st + o.off;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + c * 32, v);
+        for (int s2 = 0; s2 < sk - 1; ++s2) {
+          const uint8_t *part = sm.part[s2];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 u = *reinterpret_cast<const float4 *>(part + sk_off(lane, c * 8 + q));
+            v[4 * q] += u.x;
+            v[4 * q + 1] += u.y;
+            v[4 * q + 2] += u.z;
+            v[4 * q + 3] += u.w;
+          }
+        }
+        const int n0 = tc.nt * BN + c * 32;
+        if (row_ok && n0 < o.N) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + n0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]), pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
+                                pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]), pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]));
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncwarp();
+  // CTA 0 has received every partial before any CTA of the cluster leaves (a
+  // CTA's shared memory must outlive the copies that read or write it)
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
 }  // namespace gemm
 
 int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &a, cudaStream_t stream) {
@@ -276,7 +435,31 @@ int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &
   }
   for (int i = 0; i < 3; ++i)
     if (!P.tma_out[i]) tmO[i] = tmA;  // never read: the kernel stores problem i directly
-  const int grid = P.total_tiles < num_sms() ? P.total_tiles : num_sms();
+  // At most 32 rows and at most half as many tiles as SMs: split K over
+  // clusters of two CTAs.  Measured at M = 32, K = 12288 on B200: W_o (48
+  // tiles) 97 -> 78 us; three-CTA clusters (144 CTAs) 105 us, and launches
+  // that need a second wave (the 98-tile projections) are slower split.
+  const int sms = num_sms();
+  if (a.a_batches == 1 && a.a_rows <= SK_ROWS && SK_MAX * P.total_tiles <= sms && P.k_chunks >= 4 * SK_MAX) {
+    if (!set_smem_limit_once(reinterpret_cast<const void *>(gemm_splitk_kernel), (int)kSmemBytesSK, kSmemGemmSK))
+      return -1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(P.total_tiles * SK_MAX));
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = kSmemBytesSK;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = SK_MAX;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const CUtensorMap &s1 = a.n_problems > 1 ? tmB[1] : tmB[0];
+    const CUtensorMap &s2 = a.n_problems > 2 ? tmB[2] : tmB[0];
+    return cudaLaunchKernelEx(&cfg, gemm_splitk_kernel, tmA, tmB[0], s1, s2, P, SK_MAX) == cudaSuccess ? 0 : -1;
+  }
+  const int grid = P.total_tiles < sms ? P.total_tiles : sms;
   const CUtensorMap &b1 = a.n_problems > 1 ? tmB[1] : tmB[0];
   const CUtensorMap &b2 = a.n_problems > 2 ? tmB[2] : tmB[0];
   gemm_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB[0], b1, b2, tmO[0], tmO[1], tmO[2], P);

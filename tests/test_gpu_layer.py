@@ -53,6 +53,29 @@ def test_latent_project_matches_oracle(g, B, T, d, d_c, cache_len_max, cache_pos
     assert_parity(f64(V), orc.linear(Cr, w["W_v"]), "V")
 
 
+@pytest.mark.parametrize("B,d,d_c,cache_len_max,cache_pos", [(32, 1024, 128, 9, 5), (7, 1536, 64, 3, 2)])
+def test_decode_step_projections_split_k(g, B, d, d_c, cache_len_max, cache_pos):
+    """One new token per sequence (M = B <= 32 rows, K = d >= 768): fewer output
+    tiles than SMs, so the products run split over the K chunks by clusters of
+    CTAs whose partial rows are added in the first CTA.  Q, G, the appended
+    latent and the output projection against the oracle; cache rows other than
+    cache_pos untouched."""
+    w, t = make_layer(500 + B, B, 1, d, d_c)
+    Q = torch.empty(B, 1, d, dtype=torch.bfloat16, device="cuda")
+    G = torch.empty_like(Q)
+    C = torch.zeros(B, cache_len_max, d_c, dtype=torch.bfloat16, device="cuda")
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], None, None, Q=Q, G=G, C=C, cache_pos=cache_pos)
+    Y = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    g.gmla_gate_out(t["X"].view(B, d), t["W_o"], Y)
+    g.gmla_get_device_status()
+    assert_parity(f64(Q), orc.linear(w["X"], w["W_q"]), "Q")
+    assert_parity(f64(G), orc.linear(w["X"], w["W_g"]), "G")
+    Cg = f64(C)
+    assert_parity(Cg[:, cache_pos:cache_pos + 1], orc.linear(w["X"], w["W_c"]), "C")
+    assert np.all(Cg[:, :cache_pos] == 0) and np.all(Cg[:, cache_pos + 1:] == 0)
+    assert_parity(f64(Y), orc.linear(w["X"].reshape(B, d), w["W_o"]), "Y")
+
+
 def test_gate_out_matches_oracle(g):
     rng = np.random.default_rng(3)
     from synth_inputs import bf16_bits_from_f64
