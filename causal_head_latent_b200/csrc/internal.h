@@ -106,7 +106,7 @@ int num_sms();
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
 // device, once per (kernel slot, device): the attribute belongs to the
 // device's context, so a process that drives several GPUs sets it on each.
-enum SmemSlot { kSmemPrefill = 0, kSmemGemm = 1, kSmemLatentTc = 2, kSmemWv = 3, kSmemGemmSK = 4, kSmemSlots = 5 };
+enum SmemSlot { kSmemPrefill = 0, kSmemGemm = 1, kSmemLatentTc = 2, kSmemWv = 3, kSmemGemmSK = 4, kSmemRows = 5, kSmemSlots = 6 };
 bool set_smem_limit_once(const void *kernel, int bytes, SmemSlot slot);
 
 // bf16 TMA tensor map with 128-byte swizzle; dims/strides in elements, dim 0 contiguous.
