@@ -109,6 +109,16 @@ PROFILED_TRAFFIC = {
                            "how": "ncu dram bytes of the four kernels of one call at L=16384 (absorb, stream, merge, "
                                   "W_v); the stream kernel's cache reads (B*L*1 KB) scaled x8 to L=131072, the rest "
                                   "(q~, partial states, W_k, W_v) unscaled; profiles/gmla_attend_decode__B32_L16384.md"},
+    # decode over explicit K/V (B=8, H=96, Tk=1001): one launch at the timed size
+    "attn_rows_kernel": {"sources": ["attn_rows.cu"], "sha1": "024dbf1606e15c9acbf31d2ed3828d4eda3c3905",
+                         "bytes": 393.975296e6 + 3.392e6,
+                         "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size; "
+                                "profiles/attn_rows_kernel__B8_H96_Tk1001.md"},
+    # layer prefill: the [Q | G | C] projection, the layer's longest launch
+    "gemm_kernel": {"sources": ["gemm.cu"], "sha1": "18f16efd58b0856b99d892900ff4da2443c8d600",
+                    "bytes": 4940.081408e6 + 409.800704e6,
+                    "how": "ncu dram bytes of the [Q|G|C] projection launch of the B=2 T=4096 layer; "
+                           "profiles/gemm_kernel__layer_B2_T4096_d12288.md"},
 }
 
 
@@ -123,7 +133,7 @@ def sources_sha1(files):
 
 def profiled_traffic(kernel):
     ent = PROFILED_TRAFFIC.get(kernel)
-    if not ent or ent["bytes"] is None:
+    if not ent or ent["bytes"] is None or ent["sha1"] is None:
         return None, "no ncu capture of the current source"
     if sources_sha1(ent["sources"]) != ent["sha1"]:
         return None, "kernel changed since the ncu capture"
@@ -796,6 +806,7 @@ def main():
     if layer:
         t_l = sum(perd[k] for k in ("layer_project", "layer_attend", "layer_out")) / K
         tf = layer.flops / (t_l / 1e3) / 1e12
+        ltr, ltr_how = profiled_traffic("gemm_kernel")
         H = DM // D
         M = L_B * L_T
         parts_flops = {"layer_project": 2.0 * M * DM * (2 * DM + DC) + 2.0 * M * DC * 2 * DM,
@@ -804,7 +815,8 @@ def main():
                 "workload": f"Gated MLA layer prefill B={L_B} T={L_T} d_model={DM} H=96 D_h=128 d_c={DC}",
                 "algorithmic_flops": layer.flops,
                 "roofline": {"bound": "tensor", "achieved": tf, "peak": burst, "unit": "TFLOP/s", "frac": tf / burst,
-                             "traffic": None, "peak_kind": f"{peaks['source']} burst bf16",
+                             "traffic": ltr, "traffic_source": ltr_how, "traffic_kernel": "gemm_kernel ([Q|G|C] launch)",
+                             "peak_kind": f"{peaks['source']} burst bf16",
                              "frac_of_sustained": tf / peaks["bf16_tflops_sustained"]},
                 "clocks": region_clocks["layer"],
                 "calls": {k: {"ms": perd[k] / K, "tflops": f / (perd[k] / K / 1e3) / 1e12}
@@ -815,10 +827,12 @@ def main():
     if plain:
         t_p = perd["plain_decode"] / K
         gbs = plain.bytes / (t_p / 1e3) / 1e9
+        ptr, ptr_how = profiled_traffic("attn_rows_kernel")
         pobj = {"value": gbs * world, "unit": "GB/s", "ms_per_step": t_p,
                 "workload": f"decode attention over explicit K/V B={PL_B} H=96 Tq=1 Tk={PL_TK} D_h=128 [B,H,T,D]",
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": gbs / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": plain.bytes,
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": ptr, "traffic_source": ptr_how,
+                             "algorithmic_bytes": plain.bytes,
                              "kernel": "attn_rows_kernel", "peak_kind": f"{peaks['source']} HBM copy",
                              "l2": "394 MB of K/V, timed back to back (a step reads them once; about 3x L2)"},
                 "clocks": region_clocks["plain"]}
