@@ -272,10 +272,15 @@ GMLA_API size_t gmla_attend_decode_workspace_size(int64_t B, int64_t L, int64_t 
  *  weights optional float32 [B, H, cache_len_max]; columns at or past lens[b]
  *          are written as 0.
  *  workspace >= gmla_attend_decode_varlen_workspace_size(B, cache_len_max,
- *          H, d_c) bytes, 16-byte aligned; it also receives one tensor map and
- *          one length per sequence (copied from the host on `stream` before the
- *          launches; the call places them on a 256-byte boundary inside the
- *          workspace, which the reported size allows for).
+ *          H, d_c) bytes, 16-byte aligned; it also receives one tensor map,
+ *          one length and one record offset per sequence and the list of work
+ *          items (copied from the host on `stream` before the launches; the
+ *          call places them on 256-byte boundaries inside the workspace, which
+ *          the reported size allows for).  The rows of every sequence are cut
+ *          into work items of at most kps keys, kps chosen from `lens` on the
+ *          host, so that the thread blocks of one launch stream about equally
+ *          many latents whatever the length mix; the size depends only on
+ *          (B, cache_len_max, H, d_c).
  * Errors: GMLA_ERR_ARG for a null pointer or a length outside 1..cache_len_max,
  * the rest as gmla_attend_decode.
  */
