@@ -9,7 +9,7 @@
 //
 // One CTA owns two 128-row query tiles (Q0, Q1) of one (b, h) and streams the
 // K/V tiles they need once for both:
-//   warp 0      TMA producer: Q0, Q1, then K and V tiles into 2-stage rings
+//   warp 0      TMA producer: Q0, K0, Q1, V0, then K and V tiles into 2-stage rings
 //   warp 1      TMEM owner and MMA issuer (one thread).  Per key tile j the
 //               tensor core runs   PV0_j, S0_{j+1}, PV1_j, S1_{j+1}
 //               with S_i = Q_i K^T (both operands K-major, in shared memory)
@@ -43,7 +43,7 @@ struct Smem {
   uint8_t q[2][TILE_BYTES];
   uint8_t k[STAGES][TILE_BYTES];
   uint8_t v[STAGES][TILE_BYTES];
-  uint64_t bar_q;
+  uint64_t bar_q[2];
   uint64_t k_full[STAGES], k_empty[STAGES];
   uint64_t v_full[STAGES], v_empty[STAGES];
   uint64_t s_full[2];
@@ -125,7 +125,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (nkv == 0) return;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.bar_q, 1);
+    mbar_init(&sm.bar_q[0], 1);
+    mbar_init(&sm.bar_q[1], 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -170,11 +171,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(mk);
       tma_prefetch_desc(mv);
       const int q0 = 2 * ct * BM;
-      mbar_arrive_expect_tx(&sm.bar_q, 2 * TILE_BYTES);
-      for (int i = 0; i < 2; ++i) {
-        load(sm.q[i], mq, &sm.bar_q, 0, q0 + i * BM);
-        load(sm.q[i] + CHUNK_BYTES, mq, &sm.bar_q, 64, q0 + i * BM);
-      }
+      // Q0 and K0 first: the first S product needs only them; Q1 follows K0
+      auto load_q = [&](int i) {
+        mbar_arrive_expect_tx(&sm.bar_q[i], TILE_BYTES);
+        load(sm.q[i], mq, &sm.bar_q[i], 0, q0 + i * BM);
+        load(sm.q[i] + CHUNK_BYTES, mq, &sm.bar_q[i], 64, q0 + i * BM);
+      };
+      load_q(0);
       for (int j = 0; j < nkv; ++j) {
         const int s = j % STAGES, ph = ((j / STAGES) & 1) ^ 1;
         const int k0 = j * BN;
@@ -182,6 +185,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive_expect_tx(&sm.k_full[s], TILE_BYTES);
         load(sm.k[s], mk, &sm.k_full[s], 0, k0);
         load(sm.k[s] + CHUNK_BYTES, mk, &sm.k_full[s], 64, k0);
+        if (j == 0) load_q(1);
         if (!mbar_wait(&sm.v_empty[s], ph, p.status)) break;
         mbar_arrive_expect_tx(&sm.v_full[s], TILE_BYTES);
         load(sm.v[s], mv, &sm.v_full[s], 0, k0);
@@ -195,7 +199,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t idPV = idesc_bf16_f32(128, 128, false, true);
       const uint32_t aQ[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
       const int nk[2] = {nkv0, nkv1};
-      bool ok = mbar_wait(&sm.bar_q, 0, p.status);
+      bool ok = mbar_wait(&sm.bar_q[0], 0, p.status);
       // S_i for key tile j (K-major Q_i and K_j)
       auto issue_s = [&](int i, int j) {
         const uint32_t aK = smem_u32(sm.k[j % STAGES]);
@@ -217,8 +221,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (ok) ok = mbar_wait(&sm.k_full[0], 0, p.status);
       if (ok) {
         tc_fence_after();
-        for (int i = 0; i < 2; ++i)
-          if (nk[i] > 0) issue_s(i, 0);
+        if (nk[0] > 0) issue_s(0, 0);
+        if (nk[1] > 0) {
+          ok = mbar_wait(&sm.bar_q[1], 0, p.status);
+          tc_fence_after();
+          if (ok) issue_s(1, 0);
+        }
         umma_commit(&sm.k_empty[0]);
       }
       for (int j = 0; ok && j < nkv; ++j) {
