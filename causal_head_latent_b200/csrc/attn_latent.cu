@@ -50,97 +50,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// ---------------------------------------------------------------- absorb
-// grid (H, ceil(d_c / 128), ceil(B / AB)), 128 threads.  The CTA copies its
-// 128 x 128 tile of W_k^(h) (rows d, columns 128*y ..) and the AB query rows
-// of head h into shared memory with 16-byte loads that are all in flight at
-// once.  Thread t then owns four adjacent columns c = 128*y + 4*(t % 32) and
-// eight sequences b = b0 + 8*(t / 32) ..: per four rows d it reads four
-// 8-byte groups of W_k (adjacent lanes, adjacent addresses) and eight float4
-// of q (the same address across the warp: a broadcast) for 128 multiply-adds.
-constexpr int AB = 32;
-constexpr size_t kAbsorbSmem = AB * HD * sizeof(float) + HD * 128 * sizeof(uint16_t);  // 48 KB
-
-__global__ void __launch_bounds__(128) absorb_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ Wk,
-                                                     int B, int H, int dc, float sl2, uint16_t *__restrict__ qt) {
-  extern __shared__ __align__(16) uint8_t absorb_sm[];
-  float *qs = reinterpret_cast<float *>(absorb_sm);                      // [AB][HD]
-  uint16_t *ws = reinterpret_cast<uint16_t *>(absorb_sm + AB * HD * 4);  // [HD][128]
-  const int h = blockIdx.x, c0 = blockIdx.y * 128, b0 = blockIdx.z * AB;
-  const int nb = min(AB, B - b0);
-  const int ncol = min(128, dc - c0);  // 64 or 128 (d_c is a multiple of 64)
-  {
-    // sixteen 16-byte loads per thread, all issued before the first store
-    uint4 t[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i = threadIdx.x + 128 * k, d = i >> 4, v = i & 15;
-      t[k] = 8 * v < ncol ? *reinterpret_cast<const uint4 *>(Wk + ((size_t)h * HD + d) * dc + c0 + 8 * v)
-                          : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i = threadIdx.x + 128 * k, d = i >> 4, v = i & 15;
-      *reinterpret_cast<uint4 *>(ws + d * 128 + 8 * v) = t[k];
-    }
-  }
-  for (int i = threadIdx.x; i < AB * 16; i += 128) {
-    const int j = i >> 4, v = i & 15;
-    float *dst = qs + j * HD + 8 * v;
-    if (j < nb) {
-      const uint4 u = *reinterpret_cast<const uint4 *>(Q + (size_t)(b0 + j) * H * HD + (size_t)h * HD + 8 * v);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        dst[2 * e] = __uint_as_float(w[e] << 16);
-        dst[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dst[e] = 0.f;  // rows past B: computed, never stored
-    }
-  }
-  __syncthreads();
-  const int cq = 4 * (threadIdx.x & 31);  // first of this thread's four columns
-  const int jg = 8 * (threadIdx.x >> 5);  // first of its eight sequences
-  if (cq >= ncol) return;
-  float acc[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
-#pragma unroll 2
-  for (int d = 0; d < HD; d += 4) {
-    float w[4][4];  // [row d+e][column cq+k]
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint2 u = *reinterpret_cast<const uint2 *>(ws + (d + e) * 128 + cq);
-      w[e][0] = __uint_as_float(u.x << 16);
-      w[e][1] = __uint_as_float(u.x & 0xFFFF0000u);
-      w[e][2] = __uint_as_float(u.y << 16);
-      w[e][3] = __uint_as_float(u.y & 0xFFFF0000u);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 q4 = *reinterpret_cast<const float4 *>(qs + (jg + j) * HD + d);
-      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[j][k] = fmaf(qv[e], w[e][k], acc[j][k]);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (jg + j < nb) {
-      uint2 o;
-      o.x = pack_bf16x2(acc[j][0] * sl2, acc[j][1] * sl2);
-      o.y = pack_bf16x2(acc[j][2] * sl2, acc[j][3] * sl2);
-      *reinterpret_cast<uint2 *>(qt + ((size_t)(b0 + jg + j) * H + h) * dc + c0 + cq) = o;
-    }
-  }
-}
-
 // ---------------------------------------------------------------- combine (gmla_decode_combine)
 // Merge of n states and W_v in one kernel, for gmla_decode_combine, which has
 // no scratch for c^.  grid (H, ceil(B / CB)), CT threads.  Phase 1: warp bb
@@ -366,128 +275,6 @@ __global__ void __launch_bounds__(MT) merge_kernel(const MergeParams P) {
   }
 }
 
-// ---------------------------------------------------------------- W_v and gate (decode path)
-// o_h[b, r] = sum_c W_v[h*128 + r, c] c^[b, h, c], then the gate.  grid (H,
-// ceil(B / WV_CB)), 256 threads.  W_v^(h) (128 rows of d_c, contiguous)
-// streams through shared memory in chunks of 32 rows by 1-D bulk copies, two
-// chunks in flight; c^ of the CTA's WV_CB = 16 sequences is staged in shared
-// memory once (each head's W_v is read by ceil(B / 16) CTAs).  For each chunk,
-// warp w takes sequences b0 + 2w, b0 + 2w + 1 with lanes over columns (lane l:
-// columns 16l .. 16l+15, read as two 16-byte words per row, conflict-free) and
-// holds 32 partial sums per sequence; a transpose-reduce across the warp (31
-// shuffles per sequence) leaves lane l with the full sums of the chunk's row l.
-struct WvParams {
-  const float *chat;  // [B, H, dc]
-  const uint16_t *Wv, *G;
-  uint16_t *O;
-  int B, H, dc;
-  unsigned *status;
-};
-
-constexpr int WV_ROWS = 32;  // rows of W_v per chunk
-constexpr int WV_CB = 16;    // sequences per CTA (two per warp)
-
-__global__ void __launch_bounds__(CT) wv_kernel(const WvParams P) {
-  extern __shared__ __align__(128) uint8_t wv_sm[];
-  const int dc = P.dc;
-  const uint32_t chunk_bytes = WV_ROWS * dc * 2;
-  uint16_t *wbuf = reinterpret_cast<uint16_t *>(wv_sm);                  // [2][WV_ROWS][dc]
-  float *csm = reinterpret_cast<float *>(wv_sm + 2 * chunk_bytes);       // [WV_CB][dc]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(csm + WV_CB * dc);        // [2]
-  const int h = blockIdx.x, b0 = blockIdx.y * WV_CB;
-  const int nb = min(WV_CB, P.B - b0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NCHUNK = HD / WV_ROWS;
-  const uint16_t *wsrc = P.Wv + (size_t)h * HD * dc;
-  if (threadIdx.x == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    fence_barrier_init();
-    for (int c = 0; c < 2; ++c) {
-      mbar_arrive_expect_tx(&bar[c], chunk_bytes);
-      bulk_load(wbuf + (size_t)c * WV_ROWS * dc, wsrc + (size_t)c * WV_ROWS * dc, chunk_bytes, &bar[c]);
-    }
-  }
-  // c^ of the CTA's sequences: up to eight 16-byte loads per thread, all in flight
-  for (int base = 0; base < nb * dc / 4; base += 8 * CT) {
-    float4 t[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i4 = base + threadIdx.x + k * CT;
-      const int bb = (i4 * 4) / dc, c = (i4 * 4) % dc;
-      t[k] = i4 < nb * dc / 4 ? *reinterpret_cast<const float4 *>(P.chat + ((size_t)(b0 + bb) * P.H + h) * dc + c)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i4 = base + threadIdx.x + k * CT;
-      if (i4 < nb * dc / 4) *reinterpret_cast<float4 *>(csm + i4 * 4) = t[k];
-    }
-  }
-  __syncthreads();  // c^ staged; barrier initialisation visible
-  const int c0 = 16 * lane;
-  const bool cols_ok = c0 < dc;
-  const int bw = 2 * warp;  // this warp's first sequence within the CTA
-  float cx[2][16];
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-#pragma unroll
-    for (int e = 0; e < 16; ++e) cx[k][e] = (cols_ok && bw + k < nb) ? csm[(bw + k) * dc + c0 + e] : 0.f;
-  bool ok = true;
-#pragma unroll 1
-  for (int ch = 0; ch < NCHUNK; ++ch) {
-    const int buf = ch & 1;
-    ok = ok && mbar_wait(&bar[buf], (ch >> 1) & 1, P.status);
-    const uint16_t *wch = wbuf + (size_t)buf * WV_ROWS * dc;
-    float part[2][WV_ROWS];
-#pragma unroll
-    for (int i = 0; i < WV_ROWS; ++i) {
-      float a0 = 0.f, a1 = 0.f;
-      if (cols_ok) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(wch + (size_t)i * dc + c0);
-        const uint4 v0 = src[0], v1 = src[1];
-        const uint32_t ww[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float w0 = __uint_as_float(ww[e] << 16), w1 = __uint_as_float(ww[e] & 0xFFFF0000u);
-          a0 = fmaf(w1, cx[0][2 * e + 1], fmaf(w0, cx[0][2 * e], a0));
-          a1 = fmaf(w1, cx[1][2 * e + 1], fmaf(w0, cx[1][2 * e], a1));
-        }
-      }
-      part[0][i] = a0;
-      part[1][i] = a1;
-    }
-    __syncthreads();  // every warp has read this chunk: its buffer may be refilled
-    if (threadIdx.x == 0 && ok && ch + 2 < NCHUNK) {
-      mbar_arrive_expect_tx(&bar[buf], chunk_bytes);
-      bulk_load(wbuf + (size_t)buf * WV_ROWS * dc, wsrc + (size_t)(ch + 2) * WV_ROWS * dc, chunk_bytes, &bar[buf]);
-    }
-    // transpose-reduce: after the step with offset o each lane keeps the half
-    // of its rows whose index has lane's bit o, adding its partner's copy
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const bool up = (lane & o) != 0;
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < o; ++i) {
-          const float send = up ? part[k][i] : part[k][i + o];
-          const float keep = up ? part[k][i + o] : part[k][i];
-          part[k][i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      if (bw + k < nb && ok) {
-        const size_t oi = (size_t)(b0 + bw + k) * P.H * HD + (size_t)h * HD + ch * WV_ROWS + lane;
-        float v = part[k][0];
-        if (P.G) v *= sigmoidf_(bf16_to_f32(P.G[oi]));
-        P.O[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-      }
-    }
-  }
-}
-
 __global__ void weights_fix_kernel(float *w, const float *lse2, int BH, int L) {
   const size_t n = (size_t)BH * L;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
@@ -585,8 +372,7 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
       return -1;
   }
 
-  absorb_kernel<<<dim3(a.H, (a.dc + 127) / 128, (a.B + AB - 1) / AB), 128, kAbsorbSmem, stream>>>(
-      a.Q, a.Wk, a.B, a.H, a.dc, a.scale * kLog2e, qt);
+  if (launch_absorb_tc(a.Q, a.Wk, a.B, a.H, a.dc, a.scale * kLog2e, qt, a.status, stream) != 0) return -1;
   {
     CUtensorMap tq, tc;
     const long long dq[3] = {a.dc, a.H, a.B}, sq[2] = {a.dc, (long long)a.H * a.dc};
@@ -622,22 +408,7 @@ static int launch_attend_latent_plan(const LatentArgs &a, int S, int kps, cudaSt
     const size_t n4 = (size_t)M.BH * a.dc / 4;
     merge_kernel<<<(unsigned)((n4 + MT - 1) / MT), MT, 0, stream>>>(M);
   }
-  if (!a.out_chat) {
-    WvParams W;
-    W.chat = pacc;
-    W.Wv = a.Wv;
-    W.G = a.G;
-    W.O = a.O;
-    W.B = a.B;
-    W.H = a.H;
-    W.dc = a.dc;
-    W.status = a.status;
-    const size_t shm = 2 * (size_t)WV_ROWS * a.dc * 2 + sizeof(float) * WV_CB * a.dc + 2 * sizeof(uint64_t);
-    if (!set_smem_limit_once(reinterpret_cast<const void *>(wv_kernel),
-                             (int)(2 * WV_ROWS * 512 * 2 + sizeof(float) * WV_CB * 512 + 16), kSmemWv))
-      return -1;
-    wv_kernel<<<dim3(a.H, (a.B + WV_CB - 1) / WV_CB), CT, shm, stream>>>(W);
-  }
+  if (!a.out_chat && launch_wv_tc(pacc, a.Wv, a.G, a.O, a.B, a.H, a.dc, a.status, stream) != 0) return -1;
   if (a.weights && a.lens)
     weights_fix_varlen_kernel<<<4 * num_sms(), 256, 0, stream>>>(a.weights, lse2, lens_dev, a.H, a.B * a.H,
                                                                  a.cache_len_max);

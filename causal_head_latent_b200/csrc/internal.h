@@ -85,6 +85,12 @@ struct LatentArgs {
   float *out_lse = nullptr, *out_chat = nullptr;
 };
 int launch_attend_latent(const LatentArgs &a, cudaStream_t stream);
+// tcgen05 products around the latent decode (attn_latent_side.cu): q~ = scale*log2(e) W_k^(h)T q_h
+// ([B,H,dc] bf16) and O = sigmoid(G) (.) W_v^(h) c^ ([B,H*128] bf16); d_c a multiple of 64, <= 512.
+int launch_absorb_tc(const uint16_t *Q, const uint16_t *Wk, int B, int H, int dc, float sl2, uint16_t *qt,
+                     unsigned *status, cudaStream_t stream);
+int launch_wv_tc(const float *chat, const uint16_t *Wv, const uint16_t *G, uint16_t *O, int B, int H, int dc,
+                 unsigned *status, cudaStream_t stream);
 size_t latent_workspace_bytes(long long B, long long L, long long H, long long dc);
 size_t latent_varlen_workspace_bytes(long long B, long long cache_len_max, long long H, long long dc);
 // The state of an empty key range (lse = -inf, chat = 0).
@@ -106,7 +112,7 @@ int num_sms();
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
 // device, once per (kernel slot, device): the attribute belongs to the
 // device's context, so a process that drives several GPUs sets it on each.
-enum SmemSlot { kSmemPrefill = 0, kSmemGemm = 1, kSmemLatentTc = 2, kSmemWv = 3, kSmemGemmSK = 4, kSmemRows = 5, kSmemSlots = 6 };
+enum SmemSlot { kSmemPrefill = 0, kSmemGemm = 1, kSmemLatentTc = 2, kSmemWv = 3, kSmemGemmSK = 4, kSmemRows = 5, kSmemAbsorbTc = 6, kSmemSlots = 7 };
 bool set_smem_limit_once(const void *kernel, int bytes, SmemSlot slot);
 
 // bf16 TMA tensor map with 128-byte swizzle; dims/strides in elements, dim 0 contiguous.
