@@ -205,12 +205,16 @@ __global__ void __launch_bounds__(THREADS, 1) wv_tc_kernel(const __grid_constant
   tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v);
   const int r = 32 * warp + lane;  // row of W_v^(h): output channel 128h + r
   if (ok) {
+    // the gate logits of all 32 sequences first (their loads in flight together), then the stores
+    float gate[NB];
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+      gate[j] = (p.G && b0 + j < p.B) ? bf16_to_f32(p.G[(size_t)(b0 + j) * p.H * HD + (size_t)h * HD + r]) : 0.f;
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
       if (b0 + j < p.B) {
         const size_t oi = (size_t)(b0 + j) * p.H * HD + (size_t)h * HD + r;
-        float o = v[j];
-        if (p.G) o *= sigmoidf_(bf16_to_f32(p.G[oi]));
+        const float o = p.G ? v[j] * sigmoidf_(gate[j]) : v[j];
         p.out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
       }
     }
