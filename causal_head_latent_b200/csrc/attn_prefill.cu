@@ -343,16 +343,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float inv_l = 1.f / l;
       uint16_t *orow = p.O + (long long)b * p.o_sb + (long long)t * p.o_st + (long long)h * p.o_sh;
       const uint16_t *grow = p.G ? p.G + ((size_t)b * p.Tq + t) * (size_t)(p.H * HD) + (size_t)h * HD : nullptr;
-#pragma unroll 1
+      // the row's 128 gate logits first, all sixteen 16-byte loads in flight (loaded
+      // between the stores to O they would wait for each store, as G and O may alias)
+      uint4 g16[HD / 8];
+      if (grow && row_valid) {
+#pragma unroll
+        for (int v = 0; v < HD / 8; ++v) g16[v] = reinterpret_cast<const uint4 *>(grow)[v];
+      }
+#pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         float o[32];
         tmem_ld32(tO + c * 32, o);
         if (row_valid) {
           if (grow) {
-            const uint4 *g4 = reinterpret_cast<const uint4 *>(grow + c * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-              uint4 gv = g4[v];
+              const uint4 gv = g16[c * 4 + v];
               const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
