@@ -101,24 +101,22 @@ PROFILED_TRAFFIC = {
     "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "8560f573520ac5e265901f2abf3517519f7d0f47",
                             "bytes": 605.397504e6 + 187.000064e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
-                                   "(B=1 H=96 T=8192); profiles/attn_prefill_kernel__causal_B1_H96_T8192.md"},
+                                   "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],
                            "sha1": "445eb46b6ef14125dff64d252437109d9ff0d2ea",
                            "bytes": (542.363904e6 - 536.870912e6 + 8 * 536.870912e6) + 29.634048e6 + 13.393664e6
                                     + 56.872448e6 + 19.721728e6,
                            "how": "ncu dram bytes of the four kernels of one call at L=16384 (absorb, stream, merge, "
                                   "W_v); the stream kernel's cache reads (B*L*1 KB) scaled x8 to L=131072, the rest "
-                                  "(q~, partial states, W_k, W_v) unscaled; profiles/gmla_attend_decode__B32_L16384.md"},
+                                  "(q~, partial states, W_k, W_v) unscaled"},
     # decode over explicit K/V (B=8, H=96, Tk=1001): one launch at the timed size
     "attn_rows_kernel": {"sources": ["attn_rows.cu"], "sha1": "024dbf1606e15c9acbf31d2ed3828d4eda3c3905",
                          "bytes": 393.975296e6 + 3.392e6,
-                         "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size; "
-                                "profiles/attn_rows_kernel__B8_H96_Tk1001.md"},
+                         "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size"},
     # layer prefill: the [Q | G | C] projection, the layer's longest launch
     "gemm_kernel": {"sources": ["gemm.cu"], "sha1": "18f16efd58b0856b99d892900ff4da2443c8d600",
                     "bytes": 4940.081408e6 + 409.800704e6,
-                    "how": "ncu dram bytes of the [Q|G|C] projection launch of the B=2 T=4096 layer; "
-                           "profiles/gemm_kernel__layer_B2_T4096_d12288.md"},
+                    "how": "ncu dram bytes of the [Q|G|C] projection launch of the B=2 T=4096 layer"},
 }
 
 
