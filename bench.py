@@ -98,14 +98,14 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 # were captured (sha1 over the listed files, in order); any change makes it null until the next
 # capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "8560f573520ac5e265901f2abf3517519f7d0f47",
-                            "bytes": 605.397504e6 + 187.000064e6,
+    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "f38d9926bfef7f0bccd3dbfcc49707ac59278496",
+                            "bytes": 605.654528e6 + 186.768640e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],
-                           "sha1": "445eb46b6ef14125dff64d252437109d9ff0d2ea",
-                           "bytes": (542.363904e6 - 536.870912e6 + 8 * 536.870912e6) + 29.634048e6 + 13.393664e6
-                                    + 56.872448e6 + 19.721728e6,
+                           "sha1": "d193098045f22083a4949982f6ce7064f2fd7247",
+                           "bytes": (540.487424e6 - 536.870912e6 + 8 * 536.870912e6) + 29.391104e6 + 13.393664e6
+                                    + 56.872192e6 + 19.722240e6,
                            "how": "ncu dram bytes of the four kernels of one call at L=16384 (absorb, stream, merge, "
                                   "W_v); the stream kernel's cache reads (B*L*1 KB) scaled x8 to L=131072, the rest "
                                   "(q~, partial states, W_k, W_v) unscaled"},

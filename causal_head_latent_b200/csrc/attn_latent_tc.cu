@@ -37,7 +37,9 @@
 // soon as its probabilities are ready (releasing ring slots early) while
 // score MMAs keep the pipe busy; and the ring moves in chunk pairs, so a tile
 // costs the score thread three waits and one commit and the value thread one
-// wait and two commits.
+// wait and four commits (the value thread mostly waits for probabilities, so
+// releasing each pair as soon as its value MMAs finish costs it nothing and
+// starts the load that reuses the slot up to three blocks earlier).
 //
 //   warp 0      TMA producer: q~ once, then the latents in 64-column chunks
 //               (KT keys x 64 d_c) through the ring
@@ -76,10 +78,10 @@ constexpr int PBUF = 1;                   // P^T buffers (2: the softmax of tile
 constexpr int NSLOT = KT == 64 ? 14 : (PBUF == 2 ? 16 : 18);  // latent ring depth in chunks
 constexpr int NPAIR = NSLOT / 2;          // the ring moves in chunk pairs (one 128-row d_c block)
 constexpr int NPT = NCHUNK / 2;           // chunk pairs per tile
-constexpr int NEARLY_PAIRS = 3;           // score chunk pairs of tile j issued before the value MMAs of tile j-1
+constexpr int NEARLY_PAIRS = 2;           // chunk pairs of tile j behind the score thread's first data wait
 constexpr int NTB = 4;                    // tile-indexed barriers rotate over 4 tiles
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int kPrefetchTiles = 3;         // L2 prefetch distance of the latent stream
+constexpr int kPrefetchTiles = 2;         // L2 prefetch distance of the latent stream
 constexpr int TM_S = 0;                   // S buffers at TM_S + 64*i
 constexpr int TM_ACC = 128;               // acc^T blocks: 128 + 96*blk
 constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-path drain of copies / MMAs
@@ -88,22 +90,24 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 100 ms: error-pat
 // block i -- through NPAIR pair slots.  Pair q of tile j sits in pair slot
 // (4j + q) % NPAIR, so its previous user is pair 4j + q - NPAIR: with 9 pair
 // slots (48-key tiles) a pair of tile j-2 or j-3; with 7 (64-key tiles) pair
-// q+1 of tile j-2 for q < 3 and pair 0 of tile j-1 for q = 3.  The early pairs
-// (0..2) of tile j therefore wait only on tiles j-2 and before, whose value
-// MMAs went out while the score MMAs of tile j-1 ran, and a late pair on a
+// q+1 of tile j-2 for q < 3 and pair 0 of tile j-1 for q = 3.  A load of tile
+// j therefore waits only on tiles j-2 and before, whose value MMAs went out
+// while the score MMAs of tile j-1 ran, or (64-key tiles, pair 3) on a
 // release of tile j-1 that needs nothing of tile j.  No wait is on a later
 // tile, so the ring cannot deadlock.  The two chunks of a pair are adjacent,
 // so one MN-major descriptor with a chunk-sized leading offset spans the
 // 128-row d_c block.
 //
-// Barriers are per tile (rotating over NTB tiles), not per slot, so that a
-// tile costs the MMA thread two data waits (pairs 0..2, pair 3) and two
-// release commits (pairs 0..1 after value blocks 0..1, pairs 2..3 after
-// blocks 2..3).  A rotating barrier is never more than one phase away from
-// the phase its waiter wants: the producer arms tile j only after the
-// release of tile j-2 or j-3, by which time the MMA thread has consumed
-// tile j-NTB; the producer waits for the release of tile j-2 or j-3 only
-// after it observed the releases of tiles j-4 and earlier.
+// Barriers are per tile (rotating over NTB tiles), not per slot: a tile costs
+// the score thread two data waits (pairs 0..1, pairs 2..3) and the value
+// thread one release commit per pair, after that d_c block's value MMAs.
+// Waiting first for two pairs rather than three lets the score MMAs of a tile
+// start one pair earlier; a first wait for a single pair leaves a longer
+// second wait and measured slower.  A rotating barrier is never more than one
+// phase away from the phase its waiter wants: the producer arms tile j only
+// after a release of tile j-2 or j-3, by which time the MMA threads have
+// consumed tile j-NTB; the producer waits for a release of tile j-2 or j-3
+// only after it observed the releases of tiles j-4 and earlier.
 static_assert(NSLOT % 2 == 0 && NPAIR >= NPT + NEARLY_PAIRS, "early pairs of tile j reuse slots of tile j-2");
 static_assert(P_BYTES >= 32 * 128, "P^T buffer must cover the q~ tail");
 static_assert(PBUF == 1 || (PBUF == 2 && KT == 48), "a second P^T buffer fits next to the 48-key ring only");
@@ -200,8 +204,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *bar_q = bars;
   uint64_t *full_e = bars + 1;           // [NTB]: pairs 0..NEARLY_PAIRS-1 of tile j landed
   uint64_t *full_l = full_e + NTB;       // [NTB]: the remaining pairs of tile j landed
-  uint64_t *rel = full_l + NTB;          // [NTB][2]: pairs 2h, 2h+1 of tile j released
-  uint64_t *s_full = rel + 2 * NTB;      // [2]
+  uint64_t *rel = full_l + NTB;          // [NTB][NPT]: pair q of tile j released
+  uint64_t *s_full = rel + NPT * NTB;    // [2]
   uint64_t *s_free = s_full + 2;         // [2]: the softmax has read S buffer i
   uint64_t *p_full = s_free + 2;
   uint64_t *acc_done = p_full + 1;
@@ -241,8 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int t = 0; t < NTB; ++t) {
       mbar_init(&full_e[t], NEARLY_PAIRS);
       mbar_init(&full_l[t], NPT - NEARLY_PAIRS);
-      mbar_init(&rel[2 * t], 1);
-      mbar_init(&rel[2 * t + 1], 1);
+      for (int q = 0; q < NPT; ++q) mbar_init(&rel[NPT * t + q], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -284,9 +287,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int g = 0; g < n_pairs; ++g) {
         const int ps = g % NPAIR, j = g / NPT, q = g % NPT;
         if (q == 0) prefetch_tile(j + kPrefetchTiles);
-        if (g >= NPAIR) {  // the slot's previous pair: tile t, released with its half q' / 2
-          const int gp = g - NPAIR, t = gp / NPT, hq = (gp % NPT) / 2;
-          if (!mbar_wait(&rel[2 * (t % NTB) + hq], (t / NTB) & 1, p.status)) break;
+        if (g >= NPAIR) {  // the slot's previous pair: pair q' of tile t
+          const int gp = g - NPAIR, t = gp / NPT, qp = gp % NPT;
+          if (!mbar_wait(&rel[NPT * (t % NTB) + qp], (t / NTB) & 1, p.status)) break;
         }
         uint64_t *fb = q < NEARLY_PAIRS ? &full_e[j % NTB] : &full_l[j % NTB];
         mbar_arrive_expect_tx(fb, 2 * CCHUNK);
@@ -358,8 +361,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
                          sdesc_sw128(ap + (j % PBUF) * P_BYTES + ks * 32, 16, 1024), idPV,
                          (j > 0 || ks > 0) ? 1u : 0u);
-          // rel[.][1] also tells the softmax of tile j+1 that P^T and acc^T are free
-          if (blk & 1) umma_commit(&rel[2 * (j % NTB) + (blk >> 1)]);
+          // the last release also tells the softmax of tile j+1 that P^T and acc^T are free
+          umma_commit(&rel[NPT * (j % NTB) + blk]);
         }
         if (j == n_tiles - 1) umma_commit(acc_done);
       }
@@ -414,7 +417,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ready = got;
       if (got && j >= PBUF) {
         const int jp = j - PBUF;
-        ready = __all_sync(0xffffffffu, mbar_wait(&rel[2 * (jp % NTB) + 1], (jp / NTB) & 1, p.status));
+        ready = __all_sync(0xffffffffu, mbar_wait(&rel[NPT * (jp % NTB) + NPT - 1], (jp / NTB) & 1, p.status));
         tc_fence_after();
       }
       if (bar_or(1, 128, need || !ready)) {
@@ -425,7 +428,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (PBUF > 1 && j >= 1) {
           // the rescale below touches acc^T: the value MMAs of tile j-1 must have completed
           const int jp = j - 1;
-          const bool r1 = __all_sync(0xffffffffu, mbar_wait(&rel[2 * (jp % NTB) + 1], (jp / NTB) & 1, p.status));
+          const bool r1 = __all_sync(0xffffffffu, mbar_wait(&rel[NPT * (jp % NTB) + NPT - 1], (jp / NTB) & 1, p.status));
           if (bar_or(1, 128, !r1)) {
             ok = false;
             break;
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 size_t smem_bytes() {
-  return 1024 + Q_BYTES + PBUF * P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + 4 * NTB + 9) + 16;
+  return 1024 + Q_BYTES + PBUF * P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + (2 + NPT) * NTB + 8) + 16;
 }
 
 }  // namespace latent_tc

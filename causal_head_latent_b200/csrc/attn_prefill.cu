@@ -338,18 +338,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 
     // ---------------------------------------------------------------- epilogue
+    // The row's 128 gate logits, all sixteen 16-byte loads in flight while the
+    // last P V products finish (loaded between the stores to O they would wait
+    // for each store, as G and O may alias; each thread reads its own row first).
+    const uint16_t *grow = p.G ? p.G + ((size_t)b * p.Tq + t) * (size_t)(p.H * HD) + (size_t)h * HD : nullptr;
+    uint4 g16[HD / 8];
+    if (n_tiles > 0 && ok && grow && row_valid) {
+#pragma unroll
+      for (int v = 0; v < HD / 8; ++v) g16[v] = reinterpret_cast<const uint4 *>(grow)[v];
+    }
     if (n_tiles > 0 && ok && mbar_wait(&sm.o_done, 0, p.status)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       uint16_t *orow = p.O + (long long)b * p.o_sb + (long long)t * p.o_st + (long long)h * p.o_sh;
-      const uint16_t *grow = p.G ? p.G + ((size_t)b * p.Tq + t) * (size_t)(p.H * HD) + (size_t)h * HD : nullptr;
-      // the row's 128 gate logits first, all sixteen 16-byte loads in flight (loaded
-      // between the stores to O they would wait for each store, as G and O may alias)
-      uint4 g16[HD / 8];
-      if (grow && row_valid) {
-#pragma unroll
-        for (int v = 0; v < HD / 8; ++v) g16[v] = reinterpret_cast<const uint4 *>(grow)[v];
-      }
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         float o[32];
