@@ -103,8 +103,8 @@ PROFILED_TRAFFIC = {
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],
-                           "sha1": "d193098045f22083a4949982f6ce7064f2fd7247",
-                           "bytes": (540.487424e6 - 536.870912e6 + 8 * 536.870912e6) + 29.391104e6 + 13.393664e6
+                           "sha1": "1eb37ed88d039d19eacb38351029c5f8bce0c7dd",
+                           "bytes": (540.408320e6 - 536.870912e6 + 8 * 536.870912e6) + 29.337088e6 + 13.393664e6
                                     + 56.872192e6 + 19.722240e6,
                            "how": "ncu dram bytes of the four kernels of one call at L=16384 (absorb, stream, merge, "
                                   "W_v); the stream kernel's cache reads (B*L*1 KB) scaled x8 to L=131072, the rest "

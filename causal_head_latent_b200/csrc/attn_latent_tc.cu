@@ -26,9 +26,9 @@
 //    has completed (a relaxed poll plus fence.acq_rel costs ~90), and each
 //    tcgen05.commit ~95.
 // Tiles of KT = 48 keys (kLatentTileKeys; 64 also builds): 0.92 MMAs per key,
-// and an 18-chunk latent ring (2.25 tiles) next to the 96 KB of q~, so every
-// load of tile j reuses a slot of tile j-2 or j-3 and streams while tiles
-// j-1 and j-2 are still in use.  64-key tiles need only 0.75 MMAs per key, but
+// and a 20-chunk latent ring (2.5 tiles) next to the 96 KB of q~ and the 9 KB
+// of P^T, so every load of tile j reuses a slot of tile j-2 or j-3 and streams
+// while tiles j-1 and j-2 are still in use.  64-key tiles need only 0.75 MMAs per key, but
 // their 14-chunk ring (1.75 tiles: shared memory is full) makes the last chunk
 // pair of tile j wait for the value MMAs of tile j-1, which measured slower.
 // S is double-buffered in TMEM (2 x 64 columns next to the 384 of acc^T), so
@@ -72,10 +72,14 @@ constexpr int NUM_THREADS = 224;
 constexpr int NCHUNK = 8;                 // 64-wide d_c chunks per tile (d_c <= 512)
 constexpr int QCHUNK = HMAX * 128;        // 12 KB: one d_c chunk of q~ for 96 heads
 constexpr int Q_BYTES = NCHUNK * QCHUNK;  // 96 KB
-constexpr int P_BYTES = HMAX * 128;       // P^T: one 128-byte swizzled row (up to 64 keys) per head
+// P^T [head, key] in 8-row x 16-byte core matrices without swizzle: heads
+// 8g..8g+7 at g * P_SBO, their keys 8c..8c+7 at c * 128 within that group (no
+// padding of a head's 96-byte row of 48 keys to the 128 bytes a swizzled row takes).
+constexpr int P_SBO = (KT / 8) * 128;     // bytes per group of 8 heads
+constexpr int P_BYTES = (HMAX / 8) * P_SBO;  // 9 KB (48-key tiles) or 12 KB (64)
 constexpr int CCHUNK = KT * 128;          // one d_c chunk of a tile: KT keys x 64 d_c (6 or 8 KB)
 constexpr int PBUF = 1;                   // P^T buffers (2: the softmax of tile j waits for tile j-2's value MMAs)
-constexpr int NSLOT = KT == 64 ? 14 : (PBUF == 2 ? 16 : 18);  // latent ring depth in chunks
+constexpr int NSLOT = KT == 64 ? 14 : (PBUF == 2 ? 18 : 20);  // latent ring depth in chunks
 constexpr int NPAIR = NSLOT / 2;          // the ring moves in chunk pairs (one 128-row d_c block)
 constexpr int NPT = NCHUNK / 2;           // chunk pairs per tile
 constexpr int NEARLY_PAIRS = 2;           // chunk pairs of tile j behind the score thread's first data wait
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int ks = 0; ks < KT / 16; ++ks)
             umma_bf16_ss(tmem + TM_ACC + blk * HMAX, sdesc_sw128(cst + ks * 2048, CCHUNK, 1024),
-                         sdesc_sw128(ap + (j % PBUF) * P_BYTES + ks * 32, 16, 1024), idPV,
+                         sdesc_noswizzle(ap + (j % PBUF) * P_BYTES + ks * 256, 128, P_SBO), idPV,
                          (j > 0 || ks > 0) ? 1u : 0u);
           // the last release also tells the softmax of tile j+1 that P^T and acc^T are free
           umma_commit(&rel[NPT * (j % NTB) + blk]);
@@ -376,8 +380,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool active = quarter < 3;  // lanes 96..127 of S hold only padding rows
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     float m_used = -INFINITY, l = 0.f;
-    uint8_t *prow = sp + h * 128;
-    const int sw = h & 7;
+    uint8_t *prow = sp + (h >> 3) * P_SBO + (h & 7) * 16;
     float *wrow = (p.weights && head_ok) ? p.weights + ((size_t)b * p.H + h) * (size_t)p.w_ld : nullptr;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (active) {
 #pragma unroll
         for (int u = 0; u < KT / 8; ++u)
-          *reinterpret_cast<uint4 *>(prow + (j % PBUF) * P_BYTES + ((u ^ sw) << 4)) =
+          *reinterpret_cast<uint4 *>(prow + (j % PBUF) * P_BYTES + u * 128) =
               make_uint4(pk[u * 4 + 0], pk[u * 4 + 1], pk[u * 4 + 2], pk[u * 4 + 3]);
       }
       fence_proxy_async_smem();
@@ -521,9 +524,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-size_t smem_bytes() {
+constexpr size_t smem_bytes() {
   return 1024 + Q_BYTES + PBUF * P_BYTES + NSLOT * CCHUNK + 128 * 4 + 8 * (1 + (2 + NPT) * NTB + 8) + 16;
 }
+static_assert(smem_bytes() <= 232448, "dynamic shared memory above the 227 KB a CTA may have");
+static_assert((Q_BYTES + PBUF * P_BYTES) % 1024 == 0, "the latent ring must start on a 1024-byte boundary");
 
 }  // namespace latent_tc
 

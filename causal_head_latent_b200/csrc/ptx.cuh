@@ -261,6 +261,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor for a layout without swizzle (mode 0): 8-row x 16-byte
+// core matrices, `lbo_bytes` apart along K and `sbo_bytes` apart along M / N
+// (K-major operands).
+__device__ __forceinline__ uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with bfloat16 A and B and a
 // float32 accumulator: D format (bits 4-5) = 1, A format (7-9) = 1, B format
 // (10-12) = 1, A / B major (bits 15 / 16; 1 = MN-major), N >> 3 (17-22),
