@@ -98,8 +98,8 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 # were captured (sha1 over the listed files, in order); any change makes it null until the next
 # capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "f38d9926bfef7f0bccd3dbfcc49707ac59278496",
-                            "bytes": 605.654528e6 + 186.768640e6,
+    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "ccbb5c22a4c92ef58e2a38ddb93d93577e4a19fe",
+                            "bytes": 617.188608e6 + 187.309824e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],

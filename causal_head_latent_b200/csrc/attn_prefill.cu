@@ -23,6 +23,8 @@
 // means PV_i_j is done: the softmax may then rescale O_i (lazy: only when the
 // running max grew by more than 2^8) and overwrite P_i without further waits.
 // Tiles above the diagonal are skipped; only diagonal / tail tiles are masked.
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -38,6 +40,7 @@ constexpr int CHUNK_BYTES = TILE_BYTES / 2;
 constexpr int NUM_THREADS = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p let through unrescaled
+constexpr long long kHeadGroupBytes = 32ll << 20;  // K/V bytes of the heads one launch group covers
 
 struct Smem {
   uint8_t q[2][TILE_BYTES];
@@ -67,6 +70,7 @@ struct Params {
   const int *q_lens, *kv_lens;
   const CUtensorMap *maps;
   int n_ct;          // CTAs (256-row query pairs) per (b, h)
+  int head_group;    // (b, h) pairs per group of the launch order
   float scale_log2;  // scale * log2(e)
   unsigned *status;
 };
@@ -110,10 +114,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // Head-major CTA order (the K/V of the few heads in flight stay in L2); within
-  // a head the longest (latest) query pairs first.
-  const int bh = blockIdx.x / p.n_ct;
-  const int ct = p.causal ? (p.n_ct - 1 - blockIdx.x % p.n_ct) : (blockIdx.x % p.n_ct);
+  // Launch order: the (b, h) pairs in groups of head_group, so that the K and V
+  // of the few heads in flight stay in L2; within a group the query pairs go
+  // longest (latest) first across all of the group's heads, so that the last
+  // CTAs of the launch are short ones and no long CTA starts near the end.
+  const int BH = p.B * p.H;
+  const int per_group = p.head_group * p.n_ct;
+  const int grp = blockIdx.x / per_group, rg = blockIdx.x % per_group;
+  const int gsize = min(p.head_group, BH - grp * p.head_group);  // the last group may be smaller
+  const int ci = rg / gsize;
+  const int bh = grp * p.head_group + rg % gsize;
+  const int ct = p.causal ? (p.n_ct - 1 - ci) : ci;
   const int b = bh / p.H, h = bh % p.H;
   const int Tq = p.q_lens ? p.q_lens[b] : p.Tq;  // this sequence's query rows and keys
   const int Tk = p.kv_lens ? p.kv_lens[b] : p.Tk;
@@ -420,6 +431,10 @@ int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CU
   p.maps = a.maps;
   p.causal = a.causal;
   p.n_ct = (a.Tq + 2 * BM - 1) / (2 * BM);
+  // K and V of one head take Tk * 512 bytes: a group keeps about kHeadGroupBytes
+  // of them in flight (8 heads at 8K keys, 1 from 64K keys on).
+  const long long kv_head = (long long)a.Tk * HD * 2 * 2;
+  p.head_group = (int)std::max(1LL, std::min<long long>(16, kHeadGroupBytes / std::max(1LL, kv_head)));
   p.scale_log2 = a.scale * kLog2e;
   p.status = a.status;
   const long long grid = (long long)p.n_ct * a.B * a.H;
