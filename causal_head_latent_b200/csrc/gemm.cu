@@ -240,45 +240,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 
-// ------------------------------------------------------------------ split-K for few rows
+// ------------------------------------------------------------------ few rows
 // With at most 32 output rows (a decode step: one new token per sequence) a
 // launch of 128 x 256 tiles has fewer tiles than SMs (W_o at d_model = 12288:
-// 48), and each CTA is capped by its own TMA ingress while the others idle.
-// Here a cluster of sk CTAs shares one tile, each taking a contiguous 1/sk of
-// the K chunks; CTAs 1 .. sk-1 stage their float32 partial rows in their own
-// shared memory and send them to CTA 0 with one bulk copy each, and CTA 0 adds
-// them to its accumulator and writes the bf16 tile.  Only TMEM lanes 0..31
-// (the rows) carry data, so one epilogue warp per CTA does the work.
+// 48, the [Q | G | C] projection 98), and each CTA is capped by what it can
+// pull in while the other SMs idle.  This kernel takes tiles NB columns wide
+// (256 or 192: narrower tiles give more CTAs, each streaming fewer weight
+// rows), and with sk = 2 a cluster of two CTAs shares one tile, each taking a
+// contiguous half of the K chunks; CTA 1 stages its float32 partial rows in
+// its own shared memory and sends them to CTA 0 with one bulk copy, and CTA 0
+// adds them to its accumulator and writes the bf16 tile.  Only TMEM lanes
+// 0..31 (the rows) carry data, so one epilogue warp per CTA does the work; the
+// A loads bring in those 32 rows only, and the MMA's rows 32..127 read whatever
+// the A buffer holds there, which reaches only lanes nothing reads.
 constexpr int SK_MAX = 2;
 constexpr int SK_STAGES = 4;
 constexpr int SK_ROWS = 32;
-constexpr int SK_PART_BYTES = SK_ROWS * BN * 4;  // 32 KB: one CTA's float32 partial rows
+constexpr int SK_A_BYTES = SK_ROWS * BK * 2;  // the A box: 32 rows (4 KB) at the start of a 128-row A buffer
 
+template <int NB>
 struct SmemSK {
+  static constexpr int B_TILE = NB * BK * 2;    // 32 or 24 KB
+  static constexpr int PART = SK_ROWS * NB * 4;  // one CTA's float32 partial rows
   uint8_t a[SK_STAGES][A_BYTES];
-  uint8_t b[SK_STAGES][B_BYTES];
-  uint8_t part[SK_MAX - 1][SK_PART_BYTES];  // CTA 0: partials received; others: slot 0 stages their own
+  uint8_t b[SK_STAGES][B_TILE];
+  uint8_t part[SK_MAX - 1][PART];  // CTA 0: partials received; others: slot 0 stages their own
   uint64_t full[SK_STAGES];
   uint64_t empty[SK_STAGES];
   uint64_t acc_full;
   uint64_t recv;  // CTA 0: the partials of CTAs 1 .. SK-1 have landed
   uint32_t tmem_base;
 };
-constexpr size_t kSmemBytesSK = sizeof(SmemSK) + 1024;
+template <int NB>
+constexpr size_t smem_bytes_sk() { return sizeof(SmemSK<NB>) + 1024; }
 
-// 16-byte chunk q (of 64) of row r of a partial, swizzled so that a warp
+// 16-byte chunk q (of NB/4) of row r of a partial, swizzled so that a warp
 // whose lanes hold consecutive rows touches all banks.
-__device__ __forceinline__ uint32_t sk_off(int r, int q) { return r * (BN * 4) + ((q ^ (r & 7)) << 4); }
+template <int NB>
+__device__ __forceinline__ uint32_t sk_off(int r, int q) { return r * (NB * 4) + ((q ^ (r & 7)) << 4); }
 
+template <int NB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                        const Params P, const int sk) {
+  static_assert(NB == 256 || NB == 192, "few-row tile width");
+  constexpr uint32_t TM_COLS = 256;  // NB float32 accumulator columns, allocated as a power of two
+  using Sm = SmemSK<NB>;
   extern __shared__ uint8_t smem_raw[];
-  SmemSK &sm = *reinterpret_cast<SmemSK *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Sm &sm = *reinterpret_cast<Sm *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   unsigned *status = P.g.status;
-  const int rank = (int)cluster_ctarank();
+  const int rank = (int)cluster_ctarank();  // 0 without a cluster (sk = 1)
   const int tile = blockIdx.x / sk;
   const int kc0 = (int)((long long)P.k_chunks * rank / sk), kc1 = (int)((long long)P.k_chunks * (rank + 1) / sk);
 
@@ -289,11 +302,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.recv, 1);
-    if (rank == 0) mbar_arrive_expect_tx(&sm.recv, (uint32_t)(sk - 1) * SK_PART_BYTES);
+    if (rank == 0) mbar_arrive_expect_tx(&sm.recv, (uint32_t)(sk - 1) * Sm::PART);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, BN);
+    tmem_alloc(&sm.tmem_base, TM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -310,14 +323,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kc = kc0, g = 0; kc < kc1; ++kc, ++g) {
         const int s = g % SK_STAGES;
         if (!mbar_wait(&sm.empty[s], ((g / SK_STAGES) & 1) ^ 1, status)) break;
-        mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
+        mbar_arrive_expect_tx(&sm.full[s], SK_A_BYTES + Sm::B_TILE);
         tma_load_3d(sm.a[s], &tmA, &sm.full[s], kc * BK, P.g.a_row0, 0);
-        tma_load_2d(sm.b[s], mb, &sm.full[s], kc * BK, tc.nt * BN);
+        tma_load_2d(sm.b[s], mb, &sm.full[s], kc * BK, tc.nt * NB);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, NB, false, false);
       bool ok = true;
       for (int kc = kc0, g = 0; kc < kc1; ++kc, ++g) {
         const int s = g % SK_STAGES;
@@ -340,19 +353,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // stage this CTA's partial rows and send them to CTA 0
       uint8_t *stage = sm.part[0];
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < NB / 32; ++c) {
         float v[32];
         tmem_ld32(tmem + c * 32, v);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<float4 *>(stage + sk_off(lane, c * 8 + q)) =
+          *reinterpret_cast<float4 *>(stage + sk_off<NB>(lane, c * 8 + q)) =
               got ? make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         const uint32_t dst = mapa_shared(smem_u32(sm.part[rank - 1]), 0);
-        bulk_copy_to_peer(dst, stage, SK_PART_BYTES, mapa_shared(smem_u32(&sm.recv), 0));
+        bulk_copy_to_peer(dst, stage, Sm::PART, mapa_shared(smem_u32(&sm.recv), 0));
       }
     } else {
       const bool have = mbar_wait(&sm.recv, 0, status) && got;
@@ -361,21 +374,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool row_ok = have && t < P.g.a_rows;
       uint16_t *orow = o.out + (t / o.rows_per_b) * o.sb + (t % o.rows_per_b) * o.st + o.off;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < NB / 32; ++c) {
         float v[32];
         tmem_ld32(tmem + c * 32, v);
         for (int s2 = 0; s2 < sk - 1; ++s2) {
           const uint8_t *part = sm.part[s2];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 u = *reinterpret_cast<const float4 *>(part + sk_off(lane, c * 8 + q));
+            const float4 u = *reinterpret_cast<const float4 *>(part + sk_off<NB>(lane, c * 8 + q));
             v[4 * q] += u.x;
             v[4 * q + 1] += u.y;
             v[4 * q + 2] += u.z;
             v[4 * q + 3] += u.w;
           }
         }
-        const int n0 = tc.nt * BN + c * 32;
+        const int n0 = tc.nt * NB + c * 32;
         if (row_ok && n0 < o.N) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow + n0);
 #pragma unroll
@@ -394,15 +407,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, TM_COLS);
   }
 }
 
 }  // namespace gemm
 
-int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &a, cudaStream_t stream) {
+namespace {
+
+// Tile width and split of the few-row kernel for a launch, or nb = 0 when it
+// does not apply (more than 32 rows, several batches, short K, or more tiles
+// than SMs): the choice with the most CTAs within one wave, the wider tile on
+// a tie.  At M = 32, K = 12288 on B200: W_o 48 tiles of 256 split in two (96
+// CTAs) 68 us; the [Q | G | C] projection 98 tiles of 256 unsplit 112 us.
+// Three-CTA clusters (144 CTAs for W_o) measured 105 us, and splits that need
+// a second wave were slower.
+struct FewRowsPlan {
+  int nb = 0, sk = 0, tiles = 0;
+};
+
+FewRowsPlan few_rows_plan(const GemmArgs &a, int k_chunks, int sms) {
+  FewRowsPlan best;
+  if (a.a_batches != 1 || a.a_rows > gemm::SK_ROWS) return best;
+  for (int nb : {256, 192}) {
+    int tiles = 0;
+    for (int i = 0; i < a.n_problems; ++i) tiles += (a.prob[i].N + nb - 1) / nb;
+    for (int sk = gemm::SK_MAX; sk >= 1; --sk) {
+      if ((long long)sk * tiles > sms || k_chunks < 4 * sk) continue;
+      if (sk * tiles > best.sk * best.tiles) best = FewRowsPlan{nb, sk, tiles};
+      break;  // the largest split that fits gives this width its most CTAs
+    }
+  }
+  return best;
+}
+
+template <int NB>
+int launch_few_rows(const CUtensorMap &tmA, const CUtensorMap *tmB, gemm::Params P, int sk, SmemSlot slot,
+                    cudaStream_t stream) {
   using namespace gemm;
-  if (!set_smem_limit_once(reinterpret_cast<const void *>(gemm_kernel), (int)kSmemBytes, kSmemGemm)) return -1;
+  auto kern = gemm_splitk_kernel<NB>;
+  if (!set_smem_limit_once(reinterpret_cast<const void *>(kern), (int)smem_bytes_sk<NB>(), slot)) return -1;
+  P.n_tiles_total = 0;
+  for (int i = 0; i < 3; ++i) {
+    P.n_tiles[i] = i < P.g.n_problems ? (P.g.prob[i].N + NB - 1) / NB : 0;
+    P.n_tiles_total += P.n_tiles[i];
+  }
+  P.total_tiles = P.m_tiles * P.n_tiles_total;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(P.total_tiles * sk));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes_sk<NB>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)sk;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const CUtensorMap &b1 = P.g.n_problems > 1 ? tmB[1] : tmB[0];
+  const CUtensorMap &b2 = P.g.n_problems > 2 ? tmB[2] : tmB[0];
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB[0], b1, b2, P, sk) == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace
+
+int launch_gemm(const GemmArgs &a, cudaStream_t stream) {
+  using namespace gemm;
   Params P;
   P.g = a;
   P.m_tiles_per_b = (a.a_rows + BM - 1) / BM;
@@ -415,6 +486,25 @@ int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &
   P.total_tiles = P.m_tiles * P.n_tiles_total;
   P.k_chunks = (a.K + BK - 1) / BK;
   if (P.total_tiles <= 0 || P.k_chunks <= 0) return 0;
+  const int sms = num_sms();
+  const FewRowsPlan few = few_rows_plan(a, P.k_chunks, sms);
+  // The A map: boxes of 128 rows, or of the 32 rows the few-row kernel uses
+  // (the tile's other rows feed accumulator lanes nothing reads, so they are
+  // not loaded at all rather than filled with zeros).
+  CUtensorMap tmA;
+  const unsigned bA[3] = {(unsigned)BK, (unsigned)(few.nb ? SK_ROWS : BM), 1};
+  if (!make_tmap_bf16(&tmA, a.a, 3, a.a_dims, a.a_strides, bA)) return -1;
+  // B maps (K, N_i), one box of the tile's width in N
+  CUtensorMap tmB[3];
+  for (int i = 0; i < a.n_problems; ++i) {
+    const long long dB[2] = {a.K, a.prob[i].N}, sB[1] = {a.prob[i].w_ld};
+    const unsigned bB[2] = {(unsigned)BK, (unsigned)(few.nb ? few.nb : BN)};
+    if (!make_tmap_bf16(&tmB[i], a.prob[i].w, 2, dB, sB, bB)) return -1;
+  }
+  if (few.nb == 256) return launch_few_rows<256>(tmA, tmB, P, few.sk, kSmemGemmSK, stream);
+  if (few.nb == 192) return launch_few_rows<192>(tmA, tmB, P, few.sk, kSmemGemmSK192, stream);
+
+  if (!set_smem_limit_once(reinterpret_cast<const void *>(gemm_kernel), (int)kSmemBytes, kSmemGemm)) return -1;
   // Output maps: problem i is stored by TMA when its rows can be described as
   // a 3-D tiled map (16-byte aligned base and row / batch strides).
   CUtensorMap tmO[3];
@@ -435,30 +525,6 @@ int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &
   }
   for (int i = 0; i < 3; ++i)
     if (!P.tma_out[i]) tmO[i] = tmA;  // never read: the kernel stores problem i directly
-  // At most 32 rows and at most half as many tiles as SMs: split K over
-  // clusters of two CTAs.  Measured at M = 32, K = 12288 on B200: W_o (48
-  // tiles) 97 -> 78 us; three-CTA clusters (144 CTAs) 105 us, and launches
-  // that need a second wave (the 98-tile projections) are slower split.
-  const int sms = num_sms();
-  if (a.a_batches == 1 && a.a_rows <= SK_ROWS && SK_MAX * P.total_tiles <= sms && P.k_chunks >= 4 * SK_MAX) {
-    if (!set_smem_limit_once(reinterpret_cast<const void *>(gemm_splitk_kernel), (int)kSmemBytesSK, kSmemGemmSK))
-      return -1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(P.total_tiles * SK_MAX));
-    cfg.blockDim = dim3(NUM_THREADS);
-    cfg.dynamicSmemBytes = kSmemBytesSK;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = SK_MAX;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const CUtensorMap &s1 = a.n_problems > 1 ? tmB[1] : tmB[0];
-    const CUtensorMap &s2 = a.n_problems > 2 ? tmB[2] : tmB[0];
-    return cudaLaunchKernelEx(&cfg, gemm_splitk_kernel, tmA, tmB[0], s1, s2, P, SK_MAX) == cudaSuccess ? 0 : -1;
-  }
   const int grid = P.total_tiles < sms ? P.total_tiles : sms;
   const CUtensorMap &b1 = a.n_problems > 1 ? tmB[1] : tmB[0];
   const CUtensorMap &b2 = a.n_problems > 2 ? tmB[2] : tmB[0];

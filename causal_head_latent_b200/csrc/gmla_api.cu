@@ -194,10 +194,12 @@ static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T
   // [Q | G | C] = X [W_q; W_g; W_c]^T
   {
     GemmArgs ga{};
-    CUtensorMap tmA, tmB[3];
-    const long long dA[3] = {d_model, M, 1}, sA[2] = {d_model, M * d_model};
-    const unsigned bA[3] = {64, 128, 1};
-    if (!make_tmap_bf16(&tmA, X, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+    ga.a = X;
+    ga.a_dims[0] = d_model;
+    ga.a_dims[1] = M;
+    ga.a_dims[2] = 1;
+    ga.a_strides[0] = d_model;
+    ga.a_strides[1] = M * d_model;
     ga.a_rows = (int)M;
     ga.a_batches = 1;
     ga.a_row0 = 0;
@@ -210,10 +212,9 @@ static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T
     for (int i = 0; i < 3; ++i) {
       if (!Os[i]) continue;
       const long long N = i == 2 ? d_c : w;
-      const long long dB[2] = {d_model, N}, sB[1] = {d_model};
-      const unsigned bB[2] = {64, 256};
-      if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
       GemmOut &o = ga.prob[np];
+      o.w = Ws[i];
+      o.w_ld = d_model;
       o.out = Os[i];
       o.N = (int)N;
       if (i == 2) {  // latent rows go to cache rows [cache_pos, cache_pos + T) of each batch
@@ -230,15 +231,17 @@ static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T
       ++np;
     }
     ga.n_problems = np;
-    if (np > 0 && launch_gemm(tmA, tmB, ga, s) != 0) return GMLA_ERR_CUDA;
+    if (np > 0 && launch_gemm(ga, s) != 0) return GMLA_ERR_CUDA;
   }
   // [K | V] = C [W_k; W_v]^T, reading the bf16 latents just written to the cache
   if (K || V) {
     GemmArgs ga{};
-    CUtensorMap tmA, tmB[3];
-    const long long dA[3] = {d_c, cache_pos + T, B}, sA[2] = {d_c, cache_len_max * d_c};
-    const unsigned bA[3] = {64, 128, 1};
-    if (!make_tmap_bf16(&tmA, C, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+    ga.a = C;
+    ga.a_dims[0] = d_c;
+    ga.a_dims[1] = cache_pos + T;
+    ga.a_dims[2] = B;
+    ga.a_strides[0] = d_c;
+    ga.a_strides[1] = cache_len_max * d_c;
     ga.a_rows = (int)T;
     ga.a_batches = (int)B;
     ga.a_row0 = (int)cache_pos;
@@ -249,10 +252,9 @@ static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T
     gmla_bf16 *Os[2] = {K, V};
     for (int i = 0; i < 2; ++i) {
       if (!Os[i]) continue;
-      const long long dB[2] = {d_c, w}, sB[1] = {d_c};
-      const unsigned bB[2] = {64, 256};
-      if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
       GemmOut &o = ga.prob[np];
+      o.w = Ws[i];
+      o.w_ld = d_c;
       o.out = Os[i];
       o.N = (int)w;
       o.rows_per_b = M;
@@ -262,7 +264,7 @@ static gmla_status latent_project_heads(const gmla_bf16 *X, int64_t B, int64_t T
       ++np;
     }
     ga.n_problems = np;
-    if (launch_gemm(tmA, tmB, ga, s) != 0) return GMLA_ERR_CUDA;
+    if (launch_gemm(ga, s) != 0) return GMLA_ERR_CUDA;
   }
   return GMLA_OK;
 }
@@ -304,10 +306,12 @@ gmla_status gmla_expand_kv(const gmla_bf16 *C, int64_t B, int64_t cache_len_max,
   unsigned *st = status_ptr();
   if (!st) return GMLA_ERR_CUDA;
   GemmArgs ga{};
-  CUtensorMap tmA, tmB[3];
-  const long long dA[3] = {d_c, row0 + rows, B}, sA[2] = {d_c, cache_len_max * d_c};
-  const unsigned bA[3] = {64, 128, 1};
-  if (!make_tmap_bf16(&tmA, C, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+  ga.a = C;
+  ga.a_dims[0] = d_c;
+  ga.a_dims[1] = row0 + rows;
+  ga.a_dims[2] = B;
+  ga.a_strides[0] = d_c;
+  ga.a_strides[1] = cache_len_max * d_c;
   ga.a_rows = (int)rows;
   ga.a_batches = (int)B;
   ga.a_row0 = (int)row0;
@@ -318,10 +322,9 @@ gmla_status gmla_expand_kv(const gmla_bf16 *C, int64_t B, int64_t cache_len_max,
   gmla_bf16 *Os[2] = {K, V};
   for (int i = 0; i < 2; ++i) {
     if (!Os[i]) continue;
-    const long long dB[2] = {d_c, d_model}, sB[1] = {d_c};
-    const unsigned bB[2] = {64, 256};
-    if (!make_tmap_bf16(&tmB[np], Ws[i], 2, dB, sB, bB)) return GMLA_ERR_CUDA;
     GemmOut &o = ga.prob[np];
+    o.w = Ws[i];
+    o.w_ld = d_c;
     o.out = Os[i];
     o.N = (int)d_model;
     o.rows_per_b = B * rows;
@@ -331,7 +334,7 @@ gmla_status gmla_expand_kv(const gmla_bf16 *C, int64_t B, int64_t cache_len_max,
     ++np;
   }
   ga.n_problems = np;
-  return launch_gemm(tmA, tmB, ga, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+  return launch_gemm(ga, static_cast<cudaStream_t>(stream)) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ attention over explicit Q, K, V
@@ -645,14 +648,15 @@ static gmla_status gate_out_heads(const gmla_bf16 *O, const gmla_bf16 *G, const 
     A = gated;
   }
   GemmArgs ga{};
-  CUtensorMap tmA, tmB[3];
-  const long long dA[3] = {w, M, 1}, sA[2] = {w, M * w};
-  const unsigned bA[3] = {64, 128, 1};
-  if (!make_tmap_bf16(&tmA, A, 3, dA, sA, bA)) return GMLA_ERR_CUDA;
+  ga.a = A;
+  ga.a_dims[0] = w;
+  ga.a_dims[1] = M;
+  ga.a_dims[2] = 1;
+  ga.a_strides[0] = w;
+  ga.a_strides[1] = M * w;
   // columns 128*h0 .. 128*h1-1 of every row of W_o: a strided sub-matrix
-  const long long dB[2] = {w, d_model}, sB[1] = {d_model};
-  const unsigned bB[2] = {64, 256};
-  if (!make_tmap_bf16(&tmB[0], W_o + 128 * h0, 2, dB, sB, bB)) return GMLA_ERR_CUDA;
+  ga.prob[0].w = W_o + 128 * h0;
+  ga.prob[0].w_ld = d_model;
   ga.a_rows = (int)M;
   ga.a_batches = 1;
   ga.a_row0 = 0;
@@ -665,7 +669,7 @@ static gmla_status gate_out_heads(const gmla_bf16 *O, const gmla_bf16 *G, const 
   ga.prob[0].sb = 0;
   ga.prob[0].st = d_model;
   ga.prob[0].off = 0;
-  return launch_gemm(tmA, tmB, ga, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
+  return launch_gemm(ga, s) == 0 ? GMLA_OK : GMLA_ERR_CUDA;
 }
 
 gmla_status gmla_gate_out(const gmla_bf16 *O, const gmla_bf16 *G, const gmla_bf16 *W_o, int64_t M, int64_t d_model,

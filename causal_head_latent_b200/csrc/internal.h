@@ -52,8 +52,13 @@ struct GemmOut {
   uint16_t *out;
   long long rows_per_b, sb, st, off;
   int N;
+  const uint16_t *w;  // the B operand: N rows of K elements, w_ld elements apart
+  long long w_ld;
 };
 struct GemmArgs {
+  const uint16_t *a;     // the A operand: a 3-D array (K, rows, batches) ...
+  long long a_dims[3];   // ... of these extents (elements) ...
+  long long a_strides[2];  // ... with these row and batch strides (elements)
   int a_rows;        // rows per batch of A (rows of the A map's dimension 1 that belong to the problem)
   int a_batches;     // batches (A map dimension 2)
   int a_row0;        // first row coordinate in the A map
@@ -62,8 +67,9 @@ struct GemmArgs {
   GemmOut prob[3];
   unsigned *status;
 };
-// tmA: 3-D map (K, rows, batches), box (64, 128, 1); tmB[i]: 2-D map (K, N_i), box (64, 256).
-int launch_gemm(const CUtensorMap &tmA, const CUtensorMap *tmB, const GemmArgs &a, cudaStream_t stream);
+// The tensor maps of A (K, rows, batches) and of each B (K, N_i) are built
+// here, with boxes as tall and as wide as the tiles the launch uses.
+int launch_gemm(const GemmArgs &a, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode over the latent cache
 struct LatentArgs {
@@ -112,7 +118,7 @@ int num_sms();
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
 // device, once per (kernel slot, device): the attribute belongs to the
 // device's context, so a process that drives several GPUs sets it on each.
-enum SmemSlot { kSmemPrefill = 0, kSmemGemm = 1, kSmemLatentTc = 2, kSmemWv = 3, kSmemGemmSK = 4, kSmemRows = 5, kSmemAbsorbTc = 6, kSmemSlots = 7 };
+enum SmemSlot { kSmemPrefill = 0, kSmemGemm = 1, kSmemLatentTc = 2, kSmemWv = 3, kSmemGemmSK = 4, kSmemRows = 5, kSmemAbsorbTc = 6, kSmemGemmSK192 = 7, kSmemSlots = 8 };
 bool set_smem_limit_once(const void *kernel, int bytes, SmemSlot slot);
 
 // bf16 TMA tensor map with 128-byte swizzle; dims/strides in elements, dim 0 contiguous.

@@ -76,6 +76,52 @@ def test_decode_step_projections_split_k(g, B, d, d_c, cache_len_max, cache_pos)
     assert_parity(f64(Y), orc.linear(w["X"].reshape(B, d), w["W_o"]), "Y")
 
 
+def test_decode_step_projections_full_size(g):
+    """The decode step's products at their full size: 32 new tokens, d_model=12288,
+    d_c=512.  [Q | G | C] has 131 tiles of 192 columns (the last of the latent's
+    512 columns a partial tile) run unsplit, W_o 64 tiles of 192 split over
+    two-CTA clusters (128 CTAs).  Every row against the oracle; the appended
+    latent lands in its cache row only."""
+    B, d, d_c, cache_len_max, cache_pos = 32, 12288, 512, 6, 4
+    w, t = make_layer(SEEDS["layer_prefill"] + 1, B, 1, d, d_c)
+    Q = torch.empty(B, 1, d, dtype=torch.bfloat16, device="cuda")
+    G = torch.empty_like(Q)
+    C = torch.zeros(B, cache_len_max, d_c, dtype=torch.bfloat16, device="cuda")
+    g.gmla_latent_project(t["X"], t["W_q"], t["W_g"], t["W_c"], None, None, Q=Q, G=G, C=C, cache_pos=cache_pos)
+    Y = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+    g.gmla_gate_out(t["X"].view(B, d), t["W_o"], Y)
+    g.gmla_get_device_status()
+    del t
+    torch.cuda.empty_cache()
+    X2 = w["X"].reshape(B, d)
+    assert_parity(f64(Q).reshape(B, d), orc.linear(X2, w["W_q"]), "Q (131 tiles of 192)")
+    assert_parity(f64(G).reshape(B, d), orc.linear(X2, w["W_g"]), "G")
+    Cg = f64(C)
+    assert_parity(Cg[:, cache_pos], orc.linear(X2, w["W_c"]), "C (partial last tile)")
+    assert np.all(Cg[:, :cache_pos] == 0) and np.all(Cg[:, cache_pos + 1:] == 0)
+    assert_parity(f64(Y), orc.linear(X2, w["W_o"]), "Y (64 tiles of 192, split in two)")
+
+
+@pytest.mark.parametrize("with_v", [False, True])
+def test_expand_kv_few_rows_wide(g, with_v):
+    """A few rows of one sequence expanded to a wide d_model (16384): K alone runs
+    64 tiles of 256 columns split over two-CTA clusters, K and V together 128
+    tiles of 256 unsplit (192-column tiles would need more CTAs than SMs)."""
+    B, Lmax, d_c, d = 1, 64, 512, 16384
+    dr = Draw(37)
+    cache = dr.normal((B, Lmax, d_c))
+    Wk = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    Wv = dr.normal((d, d_c), 1 / np.sqrt(d_c))
+    row0, rows = 7, 20
+    K = torch.empty(B, rows, d, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K) if with_v else None
+    g.gmla_expand_kv(to_dev(cache), row0, rows, W_k=to_dev(Wk), W_v=to_dev(Wv) if with_v else None, K=K, V=V)
+    g.gmla_get_device_status()
+    assert_parity(f64(K), orc.linear(cache[:, row0:row0 + rows], Wk), "expanded K")
+    if with_v:
+        assert_parity(f64(V), orc.linear(cache[:, row0:row0 + rows], Wv), "expanded V")
+
+
 def test_gate_out_matches_oracle(g):
     rng = np.random.default_rng(3)
     from synth_inputs import bf16_bits_from_f64
