@@ -126,12 +126,13 @@ def test_decode_softmax_page_shape_full(g):
 
 
 @pytest.mark.parametrize("Tq,Tk", [(1, 1), (1, 2), (1, 5), (2, 16), (1, 17), (1, 129), (1, 131), (4, 193), (3, 200),
-                                   (1, 1015)])
+                                   (4, 517), (1, 768), (3, 769), (2, 1024), (1, 1015)])
 @pytest.mark.parametrize("causal", [True, False])
 def test_few_query_rows_matches_oracle(g, Tq, Tk, causal):
     """Tq <= 4 runs on the CUDA-core rows kernel.  The key counts cover tiny inputs
     and last-visible-key positions whose residue mod 64 falls on every half-warp
-    pairing (the loop must keep both half-warps of a warp together)."""
+    pairing (the loop must keep both half-warps of a warp together), and key
+    counts of 8 to 16 whole or ragged tiles (517, 768, 769, 1015, 1024)."""
     inp = prefill_qkv(61 + Tk + Tq, 2, Tq, 3, Tk=Tk, gate=True)
     O, L, W = run_prefill(g, inp, causal=causal, gate=True, lse=True, weights=True)
     ref, wref, lref = orc.attention(inp["Q"], inp["K"], inp["V"], causal=causal, want_weights=True, want_lse=True)
