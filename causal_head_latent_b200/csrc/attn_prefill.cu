@@ -297,9 +297,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < BN; ++c)
           if (k0 + c > lim) x[c] = -INFINITY;
       }
-      float mx = x[0];
+      // the row maximum as 8 independent chains joined by a tree (a single
+      // chain of BN - 1 dependent max operations is all latency)
+      float m8[8];
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      for (int i = 0; i < 8; ++i) m8[i] = x[i];
+#pragma unroll
+      for (int c = 8; c < BN; c += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], x[c + i]);
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;  // scale > 0 commutes with max
       if (wrow) {
 #pragma unroll
