@@ -98,8 +98,8 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 # were captured (sha1 over the listed files, in order); any change makes it null until the next
 # capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "ccbb5c22a4c92ef58e2a38ddb93d93577e4a19fe",
-                            "bytes": 617.188608e6 + 187.309824e6,
+    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "0e0e6f616587fe2149ee3e6d06694e4e3e2e38e8",
+                            "bytes": 620.510208e6 + 187.550720e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],
@@ -114,8 +114,8 @@ PROFILED_TRAFFIC = {
                          "bytes": 393.975296e6 + 3.392e6,
                          "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size"},
     # layer prefill: the [Q | G | C] projection, the layer's longest launch
-    "gemm_kernel": {"sources": ["gemm.cu"], "sha1": "18f16efd58b0856b99d892900ff4da2443c8d600",
-                    "bytes": 4940.081408e6 + 409.800704e6,
+    "gemm_kernel": {"sources": ["gemm.cu"], "sha1": "c14101f3204573561c7cca88530491e87af79aa5",
+                    "bytes": 4938.724864e6 + 409.714432e6,
                     "how": "ncu dram bytes of the [Q|G|C] projection launch of the B=2 T=4096 layer"},
 }
 
