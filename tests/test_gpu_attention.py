@@ -144,6 +144,19 @@ def test_few_query_rows_matches_oracle(g, Tq, Tk, causal):
     assert np.abs(w - wref).max() < 1e-4
 
 
+@pytest.mark.parametrize("B,H,T", [(1, 20, 2048), (3, 7, 1100)])
+def test_prefill_launch_groups_every_row(g, B, H, T):
+    """CTAs launch in groups of (b, h) pairs, the query pairs longest first
+    across a group.  Here B*H = 20 pairs in groups of 16 (one full group and a
+    partial one of 4), and 21 pairs of a ragged length in one group that spans
+    three sequences: every output row of every head against the oracle."""
+    inp = prefill_qkv(77 + H + T, B, T, H)
+    O, L, _ = run_prefill(g, inp, lse=True)
+    ref, lref = orc.attention(inp["Q"], inp["K"], inp["V"], want_lse=True)
+    assert_parity(f64(O), ref, "grouped launch, all rows")
+    np.testing.assert_allclose(f64(L), lref, atol=5e-4)
+
+
 def test_prefill_8k_full_size_sampled(g):
     """Causal prefill B=1, H=96, T=8192 (the timed launch), checked on sampled rows."""
     T, H = 8192, 96
