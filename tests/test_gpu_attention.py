@@ -148,8 +148,9 @@ def test_few_query_rows_matches_oracle(g, Tq, Tk, causal):
 def test_prefill_launch_groups_every_row(g, B, H, T):
     """CTAs launch in groups of (b, h) pairs, the query pairs longest first
     across a group.  Here B*H = 20 pairs in groups of 16 (one full group and a
-    partial one of 4), and 21 pairs of a ragged length in one group that spans
-    three sequences: every output row of every head against the oracle."""
+    partial one of 4), and 21 pairs of a ragged length (a group of 16 that spans
+    three sequences and a partial one of 5): every output row of every head
+    against the oracle."""
     inp = prefill_qkv(77 + H + T, B, T, H)
     O, L, _ = run_prefill(g, inp, lse=True)
     ref, lref = orc.attention(inp["Q"], inp["K"], inp["V"], want_lse=True)
