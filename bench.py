@@ -95,37 +95,63 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the dominant kernels,
 # from one ncu capture each (profiles/).  Reported only while the kernel sources are the ones that
-# were captured (sha1 over the listed files, in order); any change makes it null until the next
-# capture.
+# were captured (sha1 over the code of the listed files, in order, comments and whitespace left
+# out); any change of the code makes it null until the next capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "0e0e6f616587fe2149ee3e6d06694e4e3e2e38e8",
+    "attn_prefill_kernel": {"sources": ["attn_prefill.cu"], "sha1": "336b3dc11ee7183003e7505924018957c917a78b",
                             "bytes": 620.510208e6 + 187.550720e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],
-                           "sha1": "1eb37ed88d039d19eacb38351029c5f8bce0c7dd",
+                           "sha1": "9f2cf61be9e22857aafd74a04684d4d91b9d9c41",
                            "bytes": (540.408320e6 - 536.870912e6 + 8 * 536.870912e6) + 29.337088e6 + 13.393664e6
                                     + 56.872192e6 + 19.722240e6,
                            "how": "ncu dram bytes of the four kernels of one call at L=16384 (absorb, stream, merge, "
                                   "W_v); the stream kernel's cache reads (B*L*1 KB) scaled x8 to L=131072, the rest "
                                   "(q~, partial states, W_k, W_v) unscaled"},
     # decode over explicit K/V (B=8, H=96, Tk=1001): one launch at the timed size
-    "attn_rows_kernel": {"sources": ["attn_rows.cu"], "sha1": "024dbf1606e15c9acbf31d2ed3828d4eda3c3905",
+    "attn_rows_kernel": {"sources": ["attn_rows.cu"], "sha1": "7914ef626f5b25e912d0e76e039b93074b41d327",
                          "bytes": 393.975296e6 + 3.392e6,
                          "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size"},
     # layer prefill: the [Q | G | C] projection, the layer's longest launch
-    "gemm_kernel": {"sources": ["gemm.cu"], "sha1": "c14101f3204573561c7cca88530491e87af79aa5",
+    "gemm_kernel": {"sources": ["gemm.cu"], "sha1": "fb1d0aa150a9c74b069b87bc04ef3bfbaf895d37",
                     "bytes": 4938.724864e6 + 409.714432e6,
                     "how": "ncu dram bytes of the [Q|G|C] projection launch of the B=2 T=4096 layer"},
 }
 
 
+def code_only(text):
+    """C++/CUDA source with its comments removed and whitespace collapsed, so that
+    an edit of a comment does not count as a change of the kernel (string and
+    character literals, inline PTX included, are kept verbatim)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif text[i] in "\"'":
+            q, j = text[i], i + 1
+            while j < n and text[j] != q:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def sources_sha1(files):
+    """sha1 of the code of the listed csrc files (comments and whitespace left out)."""
     import hashlib
     h = hashlib.sha1()
     for f in files:
-        with open(os.path.join(ROOT, "causal_head_latent_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "causal_head_latent_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode("utf-8"))
     return h.hexdigest()
 
 

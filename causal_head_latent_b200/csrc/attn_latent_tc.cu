@@ -19,7 +19,9 @@
 //    and the latent stream has to stay in flight without gaps;
 //  * a tcgen05.mma with N <= 128 costs ~56-66 cycles whatever its M and N, so
 //    the MMA count per key sets the compute floor: 32 score MMAs per tile
-//    (d_c / 16, whatever KT) and 4 value MMAs per 16 keys;
+//    (d_c / 16, whatever KT) and 4 value MMAs per 16 keys (a probe without
+//    one eighth of the score MMAs ran 8 % faster: the time follows the count;
+//    the same MMAs with A read from TMEM instead ran slower);
 //  * the MMA-issuing thread must not stall: a wait on its own recent MMAs
 //    (through a barrier and another warp) drains the MMA pipe, an acquire
 //    mbarrier wait between small MMAs costs ~270 cycles even when the phase
@@ -27,10 +29,11 @@
 //    tcgen05.commit ~95.
 // Tiles of KT = 48 keys (kLatentTileKeys; 64 also builds): 0.92 MMAs per key,
 // and a 20-chunk latent ring (2.5 tiles) next to the 96 KB of q~ and the 9 KB
-// of P^T, so every load of tile j reuses a slot of tile j-2 or j-3 and streams
-// while tiles j-1 and j-2 are still in use.  64-key tiles need only 0.75 MMAs per key, but
-// their 14-chunk ring (1.75 tiles: shared memory is full) makes the last chunk
-// pair of tile j wait for the value MMAs of tile j-1, which measured slower.
+// of P^T, so every load of tile j reuses a slot of tile j-2 or j-3 and
+// streams while tiles j-1 and j-2 are still in use.  64-key tiles need only
+// 0.75 MMAs per key, but their 14-chunk ring (1.75 tiles: shared memory is
+// full) makes the last chunk pair of tile j wait for the value MMAs of tile
+// j-1, which measured slower.
 // S is double-buffered in TMEM (2 x 64 columns next to the 384 of acc^T), so
 // the score MMAs of the next tile never wait for the softmax; the score and
 // value MMAs come from two threads, so the value MMAs of a tile go out as

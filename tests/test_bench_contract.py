@@ -73,3 +73,17 @@ def test_workload_arithmetic():
     assert b.SWEEP_T == (8192, 131072, 1048576)
     for t, order in zip(b.SWEEP_T, b.SWEEP_PAGE["dot_products_per_head"]):
         assert t * (t + 1) / 2 == pytest.approx(order, rel=0.06)
+
+
+def test_traffic_records_follow_the_code_not_the_comments():
+    """The recorded DRAM traffic of a kernel is reported only while the code it
+    was captured from is unchanged: a comment or whitespace edit keeps it, any
+    change of a token (inside a string literal too) drops it."""
+    b = _load_bench()
+    src = 'int a = 1;  // note\n/* block */ asm("x // y"); char q = \'"\';\n'
+    assert b.code_only(src) == b.code_only(src.replace("note", "other note").replace("  ", " "))
+    assert b.code_only(src) != b.code_only(src.replace("a = 1", "a = 2"))
+    assert b.code_only(src) != b.code_only(src.replace("x // y", "x // z"))
+    for kernel, ent in b.PROFILED_TRAFFIC.items():
+        assert len(ent["sha1"]) == 40 and ent["bytes"] > 0, kernel
+        assert all(os.path.exists(os.path.join(ROOT, "causal_head_latent_b200", "csrc", f)) for f in ent["sources"])
