@@ -23,9 +23,8 @@
 // means PV_i_j is done: the softmax may then rescale O_i (lazy: only when the
 // running max grew by more than 2^8) and overwrite P_i without further waits.
 // Tiles above the diagonal are skipped; only diagonal / tail tiles are masked.
-#include <algorithm>
-
 #include "internal.h"
+#include "launch_plan.h"
 #include "ptx.cuh"
 
 namespace gmla {
@@ -40,7 +39,6 @@ constexpr int CHUNK_BYTES = TILE_BYTES / 2;
 constexpr int NUM_THREADS = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest p let through unrescaled
-constexpr long long kHeadGroupBytes = 32ll << 20;  // K/V bytes of the heads one launch group covers
 
 struct Smem {
   uint8_t q[2][TILE_BYTES];
@@ -118,13 +116,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // of the few heads in flight stay in L2; within a group the query pairs go
   // longest (latest) first across all of the group's heads, so that the last
   // CTAs of the launch are short ones and no long CTA starts near the end.
-  const int BH = p.B * p.H;
-  const int per_group = p.head_group * p.n_ct;
-  const int grp = blockIdx.x / per_group, rg = blockIdx.x % per_group;
-  const int gsize = min(p.head_group, BH - grp * p.head_group);  // the last group may be smaller
-  const int ci = rg / gsize;
-  const int bh = grp * p.head_group + rg % gsize;
-  const int ct = p.causal ? (p.n_ct - 1 - ci) : ci;
+  int bh, ct;
+  prefill_cta_item((int)blockIdx.x, p.B * p.H, p.n_ct, p.head_group, p.causal != 0, &bh, &ct);
   const int b = bh / p.H, h = bh % p.H;
   const int Tq = p.q_lens ? p.q_lens[b] : p.Tq;  // this sequence's query rows and keys
   const int Tk = p.kv_lens ? p.kv_lens[b] : p.Tk;
@@ -438,10 +431,7 @@ int launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CU
   p.maps = a.maps;
   p.causal = a.causal;
   p.n_ct = (a.Tq + 2 * BM - 1) / (2 * BM);
-  // K and V of one head take Tk * 512 bytes: a group keeps about kHeadGroupBytes
-  // of them in flight (8 heads at 8K keys, 1 from 64K keys on).
-  const long long kv_head = (long long)a.Tk * HD * 2 * 2;
-  p.head_group = (int)std::max(1LL, std::min<long long>(16, kHeadGroupBytes / std::max(1LL, kv_head)));
+  p.head_group = prefill_head_group(a.Tk, HD);
   p.scale_log2 = a.scale * kLog2e;
   p.status = a.status;
   const long long grid = (long long)p.n_ct * a.B * a.H;

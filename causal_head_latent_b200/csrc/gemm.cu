@@ -21,6 +21,7 @@
 // The tile order walks groups of 16 m-tiles across all n-tiles so the CTAs
 // resident at one time share A rows and B columns in L2.
 #include "internal.h"
+#include "launch_plan.h"
 #include "ptx.cuh"
 
 namespace gmla {
@@ -415,31 +416,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 namespace {
 
-// Tile width and split of the few-row kernel for a launch, or nb = 0 when it
-// does not apply (more than 32 rows, several batches, short K, or more tiles
-// than SMs): the choice with the most CTAs within one wave, the wider tile on
-// a tie.  At M = 32, K = 12288 on B200: W_o 48 tiles of 256 split in two (96
-// CTAs) 68 us; the [Q | G | C] projection 98 tiles of 256 unsplit 112 us.
-// Three-CTA clusters (144 CTAs for W_o) measured 105 us, and splits that need
-// a second wave were slower.
-struct FewRowsPlan {
-  int nb = 0, sk = 0, tiles = 0;
-};
+static_assert(gemm::SK_ROWS == kFewRowsMax && gemm::SK_MAX == kFewRowsSplitMax, "few-row plan and kernel agree");
 
-FewRowsPlan few_rows_plan(const GemmArgs &a, int k_chunks, int sms) {
-  FewRowsPlan best;
-  if (a.a_batches != 1 || a.a_rows > gemm::SK_ROWS) return best;
-  for (int nb : {256, 192}) {
-    int tiles = 0;
-    for (int i = 0; i < a.n_problems; ++i) tiles += (a.prob[i].N + nb - 1) / nb;
-    for (int sk = gemm::SK_MAX; sk >= 1; --sk) {
-      if ((long long)sk * tiles > sms || k_chunks < 4 * sk) continue;
-      if (sk * tiles > best.sk * best.tiles) best = FewRowsPlan{nb, sk, tiles};
-      break;  // the largest split that fits gives this width its most CTAs
-    }
-  }
-  return best;
-}
+// The few-row plan (launch_plan.h) measured at M = 32, K = 12288 on B200: W_o
+// in 48 tiles of 256 split in two (96 CTAs) 68 us, in 64 of 192 split in two
+// (128 CTAs) 66 us; the [Q | G | C] projection in 98 tiles of 256 112 us, in
+// 131 of 192 106 us.  Three-CTA clusters (144 CTAs for W_o) measured 105 us,
+// and splits that need a second wave were slower.
 
 template <int NB>
 int launch_few_rows(const CUtensorMap &tmA, const CUtensorMap *tmB, gemm::Params P, int sk, SmemSlot slot,
@@ -487,7 +470,9 @@ int launch_gemm(const GemmArgs &a, cudaStream_t stream) {
   P.k_chunks = (a.K + BK - 1) / BK;
   if (P.total_tiles <= 0 || P.k_chunks <= 0) return 0;
   const int sms = num_sms();
-  const FewRowsPlan few = few_rows_plan(a, P.k_chunks, sms);
+  int Ns[3] = {0, 0, 0};
+  for (int i = 0; i < a.n_problems; ++i) Ns[i] = a.prob[i].N;
+  const FewRowsPlan few = few_rows_plan(a.a_rows, a.a_batches, Ns, a.n_problems, P.k_chunks, sms);
   // The A map: boxes of 128 rows, or of the 32 rows the few-row kernel uses
   // (the tile's other rows feed accumulator lanes nothing reads, so they are
   // not loaded at all rather than filled with zeros).
