@@ -98,8 +98,8 @@ def layer_flops(B=L_B, T=L_T, d=DM, dc=DC):
 # were captured (sha1 over the code of the listed files, in order, comments and whitespace left
 # out); any change of the code makes it null until the next capture.
 PROFILED_TRAFFIC = {
-    "attn_prefill_kernel": {"sources": ["attn_prefill.cu", "launch_plan.h"], "sha1": "336b3dc11ee7183003e7505924018957c917a78b",
-                            "bytes": 620.510208e6 + 187.550720e6,
+    "attn_prefill_kernel": {"sources": ["attn_prefill.cu", "launch_plan.h"], "sha1": "a98378f246e60ba619fae741d7af6d76b1f88f43",
+                            "bytes": 620.145152e6 + 188.867072e6,
                             "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size "
                                    "(B=1 H=96 T=8192)"},
     "gmla_attend_decode": {"sources": ["attn_latent.cu", "attn_latent_tc.cu", "attn_latent_side.cu"],
@@ -114,8 +114,8 @@ PROFILED_TRAFFIC = {
                          "bytes": 393.975296e6 + 3.392e6,
                          "how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at the timed size"},
     # layer prefill: the [Q | G | C] projection, the layer's longest launch
-    "gemm_kernel": {"sources": ["gemm.cu", "launch_plan.h"], "sha1": "fb1d0aa150a9c74b069b87bc04ef3bfbaf895d37",
-                    "bytes": 4938.724864e6 + 409.714432e6,
+    "gemm_kernel": {"sources": ["gemm.cu", "launch_plan.h"], "sha1": "517f893587a228afcaa3734593b18f69703d6164",
+                    "bytes": 4931.942144e6 + 406.335488e6,
                     "how": "ncu dram bytes of the [Q|G|C] projection launch of the B=2 T=4096 layer"},
 }
 
