@@ -322,7 +322,8 @@ def test_expand_kv_row_range(g):
 
 
 @pytest.mark.parametrize("B,L,Lmax,H,d_c", [(3, 700, 700, 4, 128), (2, 1, 5, 2, 64), (1, 2049, 3000, 3, 512),
-                                             (2, 4163, 4200, 96, 512), (1, 63, 64, 1, 512)])
+                                             (2, 4163, 4200, 96, 512), (1, 63, 64, 1, 512), (33, 500, 520, 5, 512),
+                                             (70, 97, 100, 3, 192)])
 def test_attend_decode_matches_oracle(g, B, L, Lmax, H, d_c):
     d = 128 * H
     dr = Draw(300 + L)
